@@ -1,0 +1,386 @@
+"""Benchmark of the quantized-KV hot path on B200.
+
+Workload ("config D" of "Hard numbers on Qwen3.8-27B's KV cache", section "KV cache
+low-bit storage"): 1 attention layer, batch 1, 4 KV heads x 256 dims, 24 query heads
+(GQA 6), K q6_0 / V q5_0, a 2,048-token q8_0 ring. One step grows the context from 0
+to 32,768 by 32 appends of 1,024 tokens (the ring evicts and requantizes) with a decode
+step after each append. Inputs are seeded synthetic tensors (K ~ N(0,1) with 8
+outlier channels per head x8, V ~ N(0,1), q ~ N(0,1)/16), resident in HBM before the
+timed region (the e2e figure copies them from pinned host memory instead).
+
+Metric: decode attention effective HBM GB/s = algorithmic bytes a decode must read
+(packed rows, scales, ring rows, q and out) / device time of the decode calls. The
+cache fits in L2, so L2 is flushed (256 MB write) before every decode and outside the
+decode's timing. Append throughput (Mtok/s, one position of all heads' K and V) is
+reported beside it.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# workload constants
+L_, B_, H_, HQ_, D_ = 1, 1, 4, 24, 256
+CTX, CHUNK, W_ = 32768, 1024, 2048
+K_FMT, V_FMT, T_FMT = 8, 6, 10                # q6_0, q5_0, q8_0
+ROW_K, ROW_V, ROW_T = 208, 176, 272           # bytes per row at D = 256
+WORKLOAD = "config D: 1 layer, batch 1, 4 KV heads x 256, 24 q heads, K q6_0 / V q5_0, " \
+           "2048-token q8_0 ring; context 0 -> 32768 by 32 appends of 1024, decode after each"
+METRIC = "quantized-KV decode attention effective HBM GB/s (% of peak); append Mtok/s"
+
+
+def decode_bytes(n: int) -> int:
+    """Algorithmic bytes of one decode at context n: every stored row of every kv
+    head (low-bit rows below the window, ring rows inside it), plus q and out."""
+    ring = min(n, W_)
+    main = n - ring
+    rows = B_ * H_ * (main * (ROW_K + ROW_V) + ring * 2 * ROW_T)
+    return rows + 2 * B_ * HQ_ * D_ * 4
+
+
+def append_bytes(n0: int, c: int) -> int:
+    """Algorithmic bytes of appending c positions at context n0: fp32 K and V input,
+    ring writes of the positions that end in the window, ring reads of evicted rows,
+    and the low-bit rows written."""
+    n1 = n0 + c
+    in_ring = min(c, W_)                                  # new rows written to the ring
+    evicted = max(0, min(n0, n1 - W_) - max(0, n0 - W_))  # old ring rows requantized
+    direct = max(0, c - W_)                               # enter-and-leave rows
+    low = evicted + direct
+    per_bh = c * 2 * D_ * 4 + in_ring * 2 * ROW_T + evicted * 2 * ROW_T + low * (ROW_K + ROW_V)
+    return B_ * H_ * per_bh
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:12]
+
+
+DECODE_SOURCES = ["quantized_mixed_precision_qx_b200/csrc/kvq_attention.cu",
+                  "quantized_mixed_precision_qx_b200/csrc/kvq_rowio.cuh",
+                  "quantized_mixed_precision_qx_b200/csrc/kvq_internal.cuh"]
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes of the decode kernels from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = source_hash(DECODE_SOURCES)
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 3 and not line.startswith("#") and f[0] == "decode_config_d" and f[2] == want:
+            return float(f[1])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+    Q = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+        "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+        "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ oracle arm
+def oracle_sample(budget_s: float = 15.0):
+    """Time the CPU oracle on the leading steps of the same schedule until the budget
+    is spent. Returns (decode GB/s, append Mtok/s, threads, description)."""
+    import oracle as orc
+    from quantized_mixed_precision_qx_b200.synth import KVRecipe, Workload
+    wl = Workload(L_, B_, H_, HQ_, D_, CTX, KVRecipe("outlier"), seed=0)
+    threads = os.cpu_count() or 1
+    c = orc.Cache(L_, B_, H_, HQ_, D_, CTX, K_FMT, V_FMT, T_FMT, W_, threads=threads)
+    t_dec = t_app = 0.0
+    bytes_dec = 0
+    toks = 0
+    steps = 0
+    n = 0
+    t_start = time.perf_counter()
+    while n < CTX and time.perf_counter() - t_start < budget_s:
+        k = wl.kv_chunk(0, n, n + CHUNK, "k")
+        v = wl.kv_chunk(0, n, n + CHUNK, "v")
+        t0 = time.perf_counter()
+        c.append(0, k, v)
+        t_app += time.perf_counter() - t0
+        n += CHUNK
+        toks += CHUNK
+        q = wl.q_decode(0, n // CHUNK - 1)
+        t0 = time.perf_counter()
+        c.decode(0, q, 1.0)
+        t_dec += time.perf_counter() - t0
+        bytes_dec += decode_bytes(n)
+        steps += 1
+    desc = f"first {steps} of 32 (append 1024 + decode) steps of the workload, context up to {n}"
+    return bytes_dec / t_dec / 1e9, toks * B_ / t_app / 1e6, threads, desc, steps
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(max(1, args.steps)):
+        gbs, mtok, threads, desc, _ = oracle_sample(budget_s=min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+        vals.append(gbs)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "append_mtok_s": mtok}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------ CUDA arm
+def run_kvq(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from quantized_mixed_precision_qx_b200 import kvq
+    from quantized_mixed_precision_qx_b200.synth import KVRecipe, Workload
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    wl = Workload(L_, B_, H_, HQ_, D_, CTX, KVRecipe("outlier"), seed=rank)
+    k_all = torch.from_numpy(wl.kv_chunk(0, 0, CTX, "k"))        # [1][CTX][4][256]
+    v_all = torch.from_numpy(wl.kv_chunk(0, 0, CTX, "v"))
+    q_all = torch.from_numpy(np.stack([wl.q_decode(0, s) for s in range(CTX // CHUNK)]))
+    k_dev, v_dev, q_dev = k_all.to(dev), v_all.to(dev), q_all.to(dev)
+    k_chunks = [k_dev[:, i:i + CHUNK].contiguous() for i in range(0, CTX, CHUNK)]
+    v_chunks = [v_dev[:, i:i + CHUNK].contiguous() for i in range(0, CTX, CHUNK)]
+    out_dev = torch.empty(CTX // CHUNK, B_, HQ_, D_, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    cache = kvq.KVCache(L_, B_, H_, HQ_, D_, CTX, K_FMT, V_FMT, T_FMT, W_, device=dev)
+    h = cache.handle
+    ws = cache.ensure_workspace(1)
+    n_steps = CTX // CHUNK
+
+    def rebind():
+        kvq.kvq_cache_bind(h, cache.dev, cache.nbytes, stream)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2 * n_steps)]
+
+    def device_step():
+        rebind()
+        for s in range(n_steps):
+            a0, a1 = ev[2 * s]
+            a0.record(stream)
+            kvq.kvq_append(h, 0, k_chunks[s], v_chunks[s], CHUNK, stream)
+            a1.record(stream)
+            flush.fill_(s & 0xFF)
+            d0, d1 = ev[2 * s + 1]
+            d0.record(stream)
+            kvq.kvq_decode_attention(h, 0, q_dev[s], 1.0, out_dev[s], ws, ws.numel(), stream)
+            d1.record(stream)
+
+    def step_times():
+        app = sum(ev[2 * s][0].elapsed_time(ev[2 * s][1]) for s in range(n_steps)) / 1e3
+        dec = sum(ev[2 * s + 1][0].elapsed_time(ev[2 * s + 1][1]) for s in range(n_steps)) / 1e3
+        return app, dec
+
+    dec_bytes = sum(decode_bytes((s + 1) * CHUNK) for s in range(n_steps))
+    app_bytes = sum(append_bytes(s * CHUNK, CHUNK) for s in range(n_steps))
+    # launches of libkvq kernels per step: append 1 each; decode = low-bit pass (n > W),
+    # ring pass (always, W > 0) and the merge
+    launches = sum(1 + (1 if (s + 1) * CHUNK > W_ else 0) + 1 + 1 for s in range(n_steps))
+
+    for _ in range(args.warmup):
+        device_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    t_step0 = torch.cuda.Event(enable_timing=True)
+    t_step1 = torch.cuda.Event(enable_timing=True)
+    app_t = dec_t = 0.0
+    dec_per_step = []
+    torch.cuda.synchronize()
+    t_step0.record(stream)
+    for _ in range(args.steps):
+        device_step()
+        torch.cuda.synchronize()
+        a, d = step_times()
+        app_t += a
+        dec_t += d
+        dec_per_step.append(d)
+    t_step1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop()
+    step_ms = t_step0.elapsed_time(t_step1) / args.steps
+
+    # ---- end to end: pinned host inputs, copies inside the timed region
+    k_host = [c.cpu().pin_memory() for c in k_chunks]
+    v_host = [c.cpu().pin_memory() for c in v_chunks]
+    q_host = q_all.pin_memory()
+    out_host = torch.empty(n_steps, B_, HQ_, D_).pin_memory()
+    k_in = torch.empty_like(k_chunks[0])
+    v_in = torch.empty_like(v_chunks[0])
+    q_in = torch.empty(B_, HQ_, D_, device=dev)
+
+    def e2e_step():
+        rebind()
+        for s in range(n_steps):
+            k_in.copy_(k_host[s], non_blocking=True)
+            v_in.copy_(v_host[s], non_blocking=True)
+            kvq.kvq_append(h, 0, k_in, v_in, CHUNK, stream)
+            q_in.copy_(q_host[s], non_blocking=True)
+            kvq.kvq_decode_attention(h, 0, q_in, 1.0, out_dev[s], ws, ws.numel(), stream)
+            out_host[s].copy_(out_dev[s], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3 / args.steps
+    h2d = n_steps * (2 * k_chunks[0].numel() * 4 + B_ * HQ_ * D_ * 4)
+    d2h = n_steps * B_ * HQ_ * D_ * 4
+
+    # ---- max over ranks
+    t = torch.tensor([dec_t, app_t, e2e_s, step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dec_t, app_t, e2e_s, step_ms = t.tolist()
+
+    if rank != 0:
+        return
+    peak, peak_kind = read_peaks()
+    value = world * dec_bytes * args.steps / dec_t / 1e9
+    achieved = dec_bytes * args.steps / dec_t / 1e9          # per GPU
+    traffic = recorded_traffic()
+    cpu = None
+    if world == 1:
+        gbs, mtok, threads, desc, _ = oracle_sample(budget_s=15.0)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "append_mtok_s": mtok}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "l2": "flushed (256 MB write) before every decode, outside its timing",
+                   "parallelism": f"replicas x{world}"},
+        "decode_frac_of_peak": achieved / peak,
+        "append_mtok_s": world * CTX * B_ * args.steps / app_t / 1e6,
+        "append_gbs": world * app_bytes * args.steps / app_t / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "decode (split-K pass 1 + merge), per call, summed over the 32 decodes of a step",
+                     "algorithmic_bytes_per_step": dec_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * dec_bytes / e2e_s / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "decode bytes / whole step time with appends and host copies"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clock_info,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_kvq(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * kvq.h -- C ABI of libkvq: attention over a block-quantized, mixed-precision KV cache
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [KVBENCH]  "KV cache quant benchmarks: KVarN 6-bit matches q8_0, 4-bit matches q5_0"
+ *              -- cache-size column of the KLD table (block byte counts).
+ *   [HARDNUM]  "Hard numbers on Qwen3.8-27B's KV cache: q8_0 is free, K is ~2x as touchy as
+ *              V, and a 2k recent-token window makes 6/5-bit basically lossless"
+ *              -- "KV cache low-bit storage" (config D: K 6-bit, V 5-bit, last 2,048
+ *              positions in an 8-bit ring) and "Reddit reactions" (two KV paths per layer,
+ *              requantization when the window boundary moves; 32 values per token block).
+ *   [BEELLAMA] "BeeLlama.cpp v0.4.1: KVarN, KV precision tail, q2_0-q3_1 KV cache"
+ *              -- KVarN, the bf16/f16 precision tail, the q2/q3/q6 types, KV-MiB table.
+ *   [OFFLOAD]  "You can offload most of Qwen3.8-Flash-Next's KV cache to RAM with little
+ *              decode slowdown" -- decode is bound by the bytes each step reads.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named dev_* / k / v / q / out / ws are DEVICE pointers (cudaMalloc or torch
+ *    memory on the cache's device), 16-byte aligned, row-major, float32 unless stated.
+ *    host_* pointers are host memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Calls
+ *    that launch work are asynchronous on that stream; one cache handle must be used
+ *    from one stream at a time.
+ *  - The caller owns all device memory: the cache buffer, inputs, outputs and
+ *    workspace. The library owns only the host-side descriptor and allocates no
+ *    device memory.
+ *  - Every call returns a kvq_status. Arguments are validated on the host before
+ *    anything is launched: a failed call launches nothing, writes nothing and leaves
+ *    the cache length unchanged. Launch failures are reported as KVQ_ERR_CUDA.
+ *    Nothing throws across the ABI and nothing aborts the process.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,     /* bad pointer, shape, index or option */
+    KVQ_ERR_UNSUPPORTED_FMT = 2, /* format not allowed in that role */
+    KVQ_ERR_CAPACITY = 3,        /* append beyond max_ctx */
+    KVQ_ERR_CALIBRATION = 4,     /* KVarN: first append shorter than the calibration window */
+    KVQ_ERR_EMPTY = 5,           /* attention over an empty cache */
+    KVQ_ERR_ALIGNMENT = 6,       /* a device pointer is not 16-byte aligned */
+    KVQ_ERR_NOT_BOUND = 7,       /* no device buffer bound yet */
+    KVQ_ERR_CUDA = 8             /* a CUDA runtime call or launch failed */
+} kvq_status;
+
+/* Block formats. A block is 32 consecutive channels of one token row ([HARDNUM],
+ * "Reddit reactions": 32 values grouped per token).
+ *  qX_0: fp16 scale d + 32 X-bit codes, 2 + 4X bytes; value = d * (u - 2^(X-1)),
+ *        d = fp16(absmax / (2^(X-1) - 1)), codes round half away from zero, then clamp.
+ *  qX_1: fp16 scale d + fp16 min m + 32 X-bit codes, 4 + 4X bytes; value = d * u + m,
+ *        d = fp16((max - min) / (2^X - 1)), m = fp16(min).
+ *  Byte counts match [KVBENCH] (q8_0 34/64 of bf16, q6_0 26/64, q5_1 24/64) and the
+ *  [BEELLAMA] KV-MiB table. BF16 / F16 store 16-bit floats (tail formats only). */
+typedef enum kvq_fmt {
+    KVQ_Q2_0 = 0, KVQ_Q2_1 = 1, KVQ_Q3_0 = 2, KVQ_Q3_1 = 3,
+    KVQ_Q4_0 = 4, KVQ_Q4_1 = 5, KVQ_Q5_0 = 6, KVQ_Q5_1 = 7,
+    KVQ_Q6_0 = 8, KVQ_Q6_1 = 9, KVQ_Q8_0 = 10, KVQ_Q8_1 = 11,
+    KVQ_BF16 = 12, KVQ_F16 = 13, KVQ_NONE = 14
+} kvq_fmt;
+
+/* Shape of a cache. head_dim in {32, 64, 128, 256}; n_q_heads = G * n_kv_heads with
+ * 1 <= G <= 8; query head hq reads KV head hq / G. kvarn = 1 enables variance-normalised
+ * blocks ([BEELLAMA] names KVarN): per (layer, batch, kv head, channel, K|V)
+ * s = fp32(sqrt(S / T + eps)), S the fp64 sum of x^2 over the first T =
+ * kvarn_calib_tokens tokens (a power of two, 64..1024) taken as a fixed pairwise tree;
+ * blocks store x / s and are read back as s * value. */
+typedef struct kvq_layout {
+    int32_t n_layers;
+    int32_t batch;
+    int32_t n_kv_heads;
+    int32_t n_q_heads;
+    int32_t head_dim;
+    int32_t kvarn;               /* 0 or 1 */
+    int64_t max_ctx;             /* positions per (layer, batch element) */
+    int32_t kvarn_calib_tokens;  /* 512 by convention */
+    int32_t reserved;            /* must be 0 */
+    double kvarn_eps;            /* 1e-6 by convention */
+} kvq_layout;
+
+typedef struct kvq_cache kvq_cache;
+
+/* Create a host-side cache descriptor. k_fmt, v_fmt: any qX_0 / qX_1 format.
+ * tail_fmt: KVQ_NONE (W must be 0) or KVQ_Q8_0 / KVQ_BF16 / KVQ_F16 with W >= 1: the
+ * most recent W positions are kept in that format in a W-row ring and requantized to
+ * the low-bit format when they leave the window ([HARDNUM] "KV cache low-bit storage",
+ * [BEELLAMA] precision tail). kvarn with a tail: the ring holds raw values and the
+ * normalisation is applied at requantization. *out receives the handle. */
+KVQ_API kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_fmt,
+                            kvq_fmt tail_fmt, int32_t W, kvq_cache** out);
+
+/* Bytes of device memory the cache needs: the low-bit store (max_ctx rows per layer,
+ * batch element, kv head, K and V), the ring (W rows each) and the KVarN scales. Equal
+ * to the block-size closed form when every row is a multiple of 16 bytes and max_ctx,
+ * W are multiples of 16 (rows are otherwise padded to 16 bytes, regions to 256). */
+KVQ_API kvq_status kvq_cache_required_bytes(const kvq_cache* cache, size_t* bytes);
+
+/* Bind caller-owned device memory (>= required bytes, 256-byte aligned) on the current
+ * device. Zero-fills it on `stream` and resets every layer's length to 0. */
+KVQ_API kvq_status kvq_cache_bind(kvq_cache* cache, void* dev_buf, size_t bytes, void* stream);
+
+/* Free the host descriptor (never the bound device memory). NULL is accepted. */
+KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
+
+/* Quantize-on-append of n_new positions to layer `layer` (all batch elements).
+ * k, v: float32 [batch][n_new][n_kv_heads][head_dim]. Positions n..n+n_new-1 are
+ * written: those that end inside the window go to the ring in tail format (evicting
+ * and requantizing the positions they displace), the others straight to the low-bit
+ * store (with a tail: through the tail format first, so chunking never changes the
+ * stored bytes). With kvarn and no scales set, the first append must carry at least
+ * kvarn_calib_tokens positions (KVQ_ERR_CALIBRATION otherwise) and computes the
+ * scales from them first. n_new = 0 is a no-op. */
+KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const float* k, const float* v,
+                      int32_t n_new, void* stream);
+
+/* Workspace bytes for kvq_decode_attention (n_query_rows = 1) or kvq_prefill_attention
+ * (n_query_rows = n_chunk). The workspace holds per-split softmax partials. */
+KVQ_API kvq_status kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t n_query_rows, size_t* bytes);
+
+/* Decode attention (GQA) over all n cached positions of `layer`:
+ * out[b][hq] = softmax_t(scale * q[b][hq] . K~[b][hq/G][t]) . V~[b][hq/G][t], with K~, V~
+ * the dequantized cache (ring rows for the last min(n, W) positions). q, out: float32
+ * [batch][n_q_heads][head_dim]. Split-K over positions, then a fixed-order merge, so the
+ * result is bit-reproducible. ws: device workspace of >= kvq_decode_workspace_bytes(1).
+ * KVQ_ERR_EMPTY when n = 0. */
+KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const float* q, float scale,
+                                float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Causal chunked-prefill attention for the n_chunk positions just appended: chunk row i
+ * sits at position n - n_chunk + i and attends to positions <= its own over the
+ * post-append cache. q, out: float32 [batch][n_chunk][n_q_heads][head_dim].
+ * Requires 1 <= n_chunk <= n. ws: >= kvq_decode_workspace_bytes(n_chunk). */
+KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const float* q, int32_t n_chunk,
+                                 float scale, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Current number of cached positions of `layer` (host-tracked, uniform over batch). */
+KVQ_API kvq_status kvq_length(const kvq_cache* cache, int32_t layer, int64_t* n);
+
+/* KVarN only: set the channel scales of `layer` instead of calibrating. sK, sV: device
+ * float32 [batch][n_kv_heads][head_dim], all > 0. Must come before the layer's first append. */
+KVQ_API kvq_status kvq_set_channel_scales(kvq_cache* cache, int32_t layer, const float* sK, const float* sV,
+                                  void* stream);
+
+/* Copy stored rows to host memory in the canonical serialisation (per 32-value block:
+ * fp16 d | [fp16 m] | code planes low bits first, little endian; BF16/F16: 32 x 2 bytes).
+ * region 0: low-bit store rows pos0..pos0+count-1; region 1: ring slots pos0..+count-1
+ * (tail format). kv: 0 = K, 1 = V. Synchronises the device. host_dst must hold
+ * count * (head_dim / 32) * block bytes. */
+KVQ_API kvq_status kvq_export_blocks(const kvq_cache* cache, int32_t layer, int32_t b, int32_t h, int32_t kv,
+                             int32_t region, int64_t pos0, int64_t count, void* host_dst, size_t bytes);
+
+/* Static description of a status code. */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -1,0 +1,255 @@
+// kvq_append.cu -- quantize-on-append, tail-ring eviction with requantization, and the
+// KVarN channel-statistics pass.
+//
+// One warp owns one (position, batch, kv head, K|V) row of D = 32*CPL channels; lane l
+// holds channels [l*CPL, (l+1)*CPL), so a 32-value block spans 32/CPL lanes and its
+// max / min reduce with xor shuffles inside that lane group. Inputs are read with
+// 16-byte loads, codes are packed in registers and written as whole words per lane.
+//
+// Block rules ([HARDNUM] "Reddit reactions": 32 values per token block; byte counts
+// from the [KVBENCH] cache-size table):
+//   qX_0: d = fp16(absmax / (2^(X-1)-1)) (saturating), q = clamp(rhaz(x / d)), u = q + 2^(X-1)
+//   qX_1: d = fp16((max - min) / (2^X - 1)), m = fp16(min), u = clamp(rhaz((x - m) / d))
+// with IEEE float32 division (__fdiv_rn) and round-half-away-from-zero (roundf).
+//
+// Ring ([HARDNUM] "KV cache low-bit storage": the last 2,048 positions in an 8-bit ring;
+// [BEELLAMA] precision tail): after an append of C rows to a cache of n, positions
+// [n+C-W, n+C) sit in ring slot pos mod W. A new position that ends inside the window
+// takes its slot: the warp first requantizes the slot's old occupant (the unique
+// position q in [n-W, n) with q = pos mod W) into the low-bit store, then writes the new
+// row. Every evicted position's slot receives exactly one such new row, and slots are
+// distinct across warps, so no two warps touch one slot. Positions that enter and leave
+// within the append go to the low-bit store directly, through the tail rounding.
+#include "kvq_rowio.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int WARPS_PER_CTA = 8;
+
+template <int CPL>
+struct Lanes {
+    static constexpr int LPB = 32 / CPL;   // lanes per 32-value block
+};
+
+// Quantize this lane's CPL values into row `row` of format f (all lanes participate).
+template <int CPL>
+__device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFmt& f, int lane,
+                                          const float (&x)[CPL]) {
+    constexpr int LPB = Lanes<CPL>::LPB;
+    if (f.kind != 0) {
+        uint16_t h[CPL];
+#pragma unroll
+        for (int j = 0; j < CPL; ++j)
+            h[j] = (f.kind == 1) ? __bfloat16_as_ushort(__float2bfloat16_rn(x[j]))
+                                 : __half_as_ushort(__float2half_rn(x[j]));
+        uint16_t* dst = reinterpret_cast<uint16_t*>(row) + lane * CPL;
+        if constexpr (CPL == 8) {
+            uint4 w;
+            w.x = h[0] | ((uint32_t)h[1] << 16); w.y = h[2] | ((uint32_t)h[3] << 16);
+            w.z = h[4] | ((uint32_t)h[5] << 16); w.w = h[6] | ((uint32_t)h[7] << 16);
+            *reinterpret_cast<uint4*>(dst) = w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) dst[j] = h[j];
+        }
+        return;
+    }
+    const int blk = (lane * CPL) >> 5;
+    uint32_t u[CPL];
+    uint16_t dh, mh = 0;
+    if (!f.asym) {
+        const int qmax = (1 << (f.bits - 1)) - 1;
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
+        a = group_max<LPB>(a);
+        const float d32 = __fdiv_rn(a, (float)qmax);
+        dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
+        const float d = __half2float(__ushort_as_half(dh));
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            float r = 0.f;
+            if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(x[j], d)), (float)-qmax), (float)qmax);
+            u[j] = (uint32_t)((int)r + qmax + 1);
+        }
+    } else {
+        const int umax = (1 << f.bits) - 1;
+        float lo = x[0], hi = x[0];
+#pragma unroll
+        for (int j = 1; j < CPL; ++j) { lo = fminf(lo, x[j]); hi = fmaxf(hi, x[j]); }
+        lo = group_min<LPB>(lo);
+        hi = group_max<LPB>(hi);
+        const float d32 = __fdiv_rn(__fsub_rn(hi, lo), (float)umax);
+        dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
+        mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
+        const float d = __half2float(__ushort_as_half(dh));
+        const float m = __half2float(__ushort_as_half(mh));
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            float r = 0.f;
+            if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(__fsub_rn(x[j], m), d)), 0.f), (float)umax);
+            u[j] = (uint32_t)r;
+        }
+    }
+    uint64_t v0 = 0, v1 = 0;
+    const uint32_t m0 = (1u << f.w0) - 1;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        v0 |= (uint64_t)(u[j] & m0) << (j * f.w0);
+        if (f.w1) v1 |= (uint64_t)(u[j] >> f.w0) << (j * f.w1);
+    }
+    store_plane_bits(row + f.off_p0, lane, CPL * f.w0, v0);
+    if (f.w1) store_plane_bits(row + f.off_p1, lane, CPL * f.w1, v1);
+    if ((lane % LPB) == 0) {
+        reinterpret_cast<uint16_t*>(row)[blk] = dh;
+        if (f.asym) reinterpret_cast<uint16_t*>(row + f.off_m)[blk] = mh;
+    }
+}
+
+// Low-bit store of a raw row (KVarN: divide by the channel scales first).
+template <int CPL>
+__device__ __forceinline__ void store_low(uint8_t* row, const RowFmt& f, const float* __restrict__ s, int lane,
+                                          float (&x)[CPL]) {
+    if (s) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) x[j] = __fdiv_rn(x[j], s[lane * CPL + j]);
+    }
+    store_row<CPL>(row, f, lane, x);
+}
+
+template <int CPL>
+__global__ void __launch_bounds__(32 * WARPS_PER_CTA)
+append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, long long n, int C) {
+    const int lane = threadIdx.x & 31;
+    const long long item = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+    const long long items = (long long)C * lv.B * lv.H * 2;
+    if (item >= items) return;
+    // item order: (b, i, h, kv) so consecutive warps read consecutive input rows
+    const int kv = (int)(item & 1);
+    const int h = (int)((item >> 1) % lv.H);
+    const long long bi = (item >> 1) / lv.H;
+    const int i = (int)(bi % C);
+    const int b = (int)(bi / C);
+    const int D = lv.D;
+    const float* src = (kv ? v : k) + (((long long)b * C + i) * lv.H + h) * D;
+    const RowFmt& fl = lv.fmt[kv];
+    uint8_t* main = lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv];
+    const float* s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * D : nullptr;
+    const long long p = n + i;
+
+    float x[CPL];
+    load_row_f32<CPL>(src, lane, x);
+
+    if (lv.W == 0) {
+        store_low<CPL>(main + p * fl.stride, fl, s, lane, x);
+        return;
+    }
+    const long long W = lv.W;
+    if (p < n + C - W) {
+        // enters and leaves the window inside this append: tail rounding, then low-bit
+        float t[CPL];
+        // round through the tail format in registers (same values a ring round trip gives)
+        if (lv.tail.kind == 1) {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) t[j] = __bfloat162float(__float2bfloat16_rn(x[j]));
+        } else if (lv.tail.kind == 2) {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) t[j] = __half2float(__float2half_rn(x[j]));
+        } else {
+            // q8_0 tail: symmetric 8-bit block quantization then exact dequantization
+            constexpr int LPB = Lanes<CPL>::LPB;
+            float a = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
+            a = group_max<LPB>(a);
+            const float d32 = __fdiv_rn(a, 127.f);
+            const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                float r = 0.f;
+                if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(x[j], d)), -127.f), 127.f);
+                t[j] = __fmul_rn(d, r);
+            }
+        }
+        store_low<CPL>(main + p * fl.stride, fl, s, lane, t);
+        return;
+    }
+    // ends inside the window: evict the slot's old occupant, then take the slot
+    uint8_t* ring = lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region;
+    const long long slot = p % W;
+    uint8_t* srow = ring + slot * lv.tail.stride;
+    const long long base = n - W;                       // old window start (may be < 0)
+    const long long q = base + ((slot - base) % W + W) % W;
+    if (q >= 0) {
+        float y[CPL];
+        load_row_values<CPL>(srow, lv.tail, lane, y);
+        __syncwarp();
+        store_low<CPL>(main + q * fl.stride, fl, s, lane, y);
+    }
+    __syncwarp();
+    store_row<CPL>(srow, lv.tail, lane, x);
+}
+
+// KVarN statistics: one CTA of T/2 threads per (b, h, K|V, channel group of 8);
+// S_c = fixed pairwise tree over a[t] = x_t^2 (a[t] += a[t + stride], stride = T/2 .. 1)
+// in float64; s_c = float(sqrt(S_c / T + eps)).
+__global__ void calibrate_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v,
+                                 int C, int T, double eps) {
+    extern __shared__ double sm[];                      // [T/2][8]
+    const int groups = lv.D / 8;
+    const int g = blockIdx.x % groups;
+    const int kv = (blockIdx.x / groups) & 1;
+    const int bh = blockIdx.x / groups / 2;
+    const int h = bh % lv.H, b = bh / lv.H;
+    const float* x = kv ? v : k;
+    const int t = threadIdx.x;                          // 0 .. T/2-1
+    const int half = T / 2;
+    const long long rs = (long long)lv.H * lv.D;
+    const float* r0 = x + ((long long)b * C + t) * rs + (long long)h * lv.D + g * 8;
+    const float* r1 = r0 + (long long)half * rs;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const double a0 = (double)r0[c], a1 = (double)r1[c];
+        sm[t * 8 + c] = __dadd_rn(__dmul_rn(a0, a0), __dmul_rn(a1, a1));
+    }
+    __syncthreads();
+    for (int stride = half / 2; stride >= 1; stride >>= 1) {
+        if (t < stride) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sm[t * 8 + c] = __dadd_rn(sm[t * 8 + c], sm[(t + stride) * 8 + c]);
+        }
+        __syncthreads();
+    }
+    if (t < 8) {
+        const double mean = __dadd_rn(sm[t] / (double)T, eps);
+        lv.scales[((long long)(b * lv.H + h) * 2 + kv) * lv.D + g * 8 + t] = __double2float_rn(sqrt(mean));
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
+                          cudaStream_t st) {
+    const long long items = (long long)C * lv.B * lv.H * 2;
+    const unsigned grid = (unsigned)((items + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
+    const dim3 block(32 * WARPS_PER_CTA);
+    switch (lv.D / 32) {
+        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
+        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
+        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
+        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calibrate(const LayerView& lv, const float* k, const float* v, int C, int T,
+                             double eps, cudaStream_t st) {
+    const unsigned grid = (unsigned)(lv.B * lv.H * 2 * (lv.D / 8));
+    const size_t smem = (size_t)(T / 2) * 8 * sizeof(double);
+    calibrate_kernel<<<grid, T / 2, smem, st>>>(lv, k, v, C, T, eps);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

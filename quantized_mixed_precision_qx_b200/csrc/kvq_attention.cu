@@ -1,0 +1,273 @@
+// kvq_attention.cu -- split-K flash-decoding over the quantized cache (decode, and the
+// row-batched form used for chunked prefill), plus the fixed-order merge.
+//
+// Decode reads every cached byte once per step, so it is bound by HBM bytes ([OFFLOAD]:
+// each decode step streams the whole attention state; the bytes read per step set the
+// token rate). Pass 1: one CTA per (split, kv head, batch x query row) streams its rows,
+// dequantizes in registers, and keeps an online softmax (running max m, sum l, output
+// accumulator o) for the G query heads that share the KV head. Low-bit rows and ring
+// rows are separate launches over separate split ranges. Pass 2 merges the splits in a
+// fixed order, so results are bit-reproducible run to run.
+//
+// Scores are kept in base-2 units: q is pre-multiplied by scale * log2(e), so
+// p = exp2(s - m) equals exp(scale * q.k - max).
+#include "kvq_rowio.cuh"
+
+#include <cfloat>
+
+namespace kvq {
+namespace {
+
+constexpr int P1_WARPS = 4;
+constexpr int MAXG = 8;
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct P1Args {
+    LayerView lv;
+    const float* q;        // [B][rows][Hq][D]
+    float qscale;          // scale * log2(e)
+    float* ws;             // partials
+    long long n;           // cached positions
+    long long pos_base;    // position of query row 0
+    int rows;
+    int ring;              // 0: low-bit rows, 1: ring rows
+    long long chunk;       // rows per split of this region
+    long long region_rows; // rows of this region (n_main or n_ring)
+    int split_offset;      // first split index of this region
+    int n_split;           // total splits per (b, row, h)
+};
+
+template <int CPL>
+__global__ void __launch_bounds__(32 * P1_WARPS)
+attn_pass1(P1Args a) {
+    const LayerView& lv = a.lv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int D = lv.D, G = lv.G, H = lv.H;
+    const int h = blockIdx.y;
+    const int br = blockIdx.z;                 // b * rows + r
+    const int b = br / a.rows, r = br % a.rows;
+    const int split = blockIdx.x;
+    const long long limit = a.pos_base + r;    // last position this row may see
+
+    const long long t0 = (long long)split * a.chunk;
+    long long t1 = t0 + a.chunk;
+    if (t1 > a.region_rows) t1 = a.region_rows;
+    if (!a.ring && t1 > limit + 1) t1 = limit + 1;   // main rows: index == position
+
+    const int kvarn = lv.kvarn && !a.ring;
+    const float* sK = kvarn ? lv.scales + ((long long)(b * H + h) * 2 + 0) * D : nullptr;
+    const float* sV = kvarn ? lv.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
+
+    // q for the G heads of this kv head, this lane's channels, pre-scaled
+    float qr[MAXG][CPL];
+    const float* qb = a.q + ((long long)br * lv.G * H + (long long)h * G) * D;
+#pragma unroll
+    for (int g = 0; g < MAXG; ++g) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const int c = lane * CPL + j;
+            float v = (g < G) ? qb[(long long)g * D + c] * a.qscale : 0.f;
+            if (kvarn) v *= sK[c];
+            qr[g][j] = v;
+        }
+    }
+
+    const RowFmt fk = a.ring ? lv.tail : lv.fmt[0];
+    const RowFmt fv = a.ring ? lv.tail : lv.fmt[1];
+    const uint8_t* kbase = a.ring ? lv.ring[0] + (long long)(b * H + h) * lv.ring_region
+                                  : lv.main[0] + (long long)(b * H + h) * lv.main_region[0];
+    const uint8_t* vbase = a.ring ? lv.ring[1] + (long long)(b * H + h) * lv.ring_region
+                                  : lv.main[1] + (long long)(b * H + h) * lv.main_region[1];
+    const long long ring_base = a.n - lv.W;    // ring slot s holds position ring_base + ((s - ring_base) mod W)
+
+    float m[MAXG], l[MAXG], o[MAXG][CPL];
+#pragma unroll
+    for (int g = 0; g < MAXG; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) o[g][j] = 0.f;
+    }
+
+    for (long long t = t0 + warp; t < t1; t += P1_WARPS) {
+        if (a.ring) {
+            const long long W = lv.W;
+            const long long pos = ring_base + ((t - ring_base) % W + W) % W;
+            if (pos > limit) continue;
+        }
+        float kx[CPL], vx[CPL];
+        load_row_values<CPL>(kbase + t * fk.stride, fk, lane, kx);
+        load_row_values<CPL>(vbase + t * fv.stride, fv, lane, vx);
+        float s[MAXG];
+#pragma unroll
+        for (int g = 0; g < MAXG; ++g) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) acc = fmaf(qr[g][j], kx[j], acc);
+            s[g] = acc;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+#pragma unroll
+            for (int g = 0; g < MAXG; ++g)
+                if (g < G) s[g] += __shfl_xor_sync(0xffffffffu, s[g], off);
+        }
+#pragma unroll
+        for (int g = 0; g < MAXG; ++g) {
+            if (g >= G) break;
+            if (s[g] > m[g]) {
+                const float corr = exp2f(m[g] - s[g]);
+                l[g] *= corr;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) o[g][j] *= corr;
+                m[g] = s[g];
+            }
+            const float p = exp2f(s[g] - m[g]);
+            l[g] += p;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) o[g][j] = fmaf(p, vx[j], o[g][j]);
+        }
+    }
+
+    // combine the warps of this CTA
+    __shared__ float sm_m[P1_WARPS][MAXG], sm_l[P1_WARPS][MAXG];
+    extern __shared__ float sm_o[];            // [P1_WARPS][G][D]
+    if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < MAXG; ++g) { sm_m[warp][g] = m[g]; sm_l[warp][g] = l[g]; }
+    }
+#pragma unroll
+    for (int g = 0; g < MAXG; ++g) {
+        if (g >= G) break;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) sm_o[((warp * G) + g) * D + lane * CPL + j] = o[g][j];
+    }
+    __syncthreads();
+
+    float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, c = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < P1_WARPS; ++w) M = fmaxf(M, sm_m[w][g]);
+        float O = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < P1_WARPS; ++w) {
+                const float e = exp2f(sm_m[w][g] - M);
+                O = fmaf(sm_o[((w * G) + g) * D + c], e, O);
+                L = fmaf(sm_l[w][g], e, L);
+            }
+        }
+        if (sV) O *= sV[c];
+        part[2 * G + idx] = O;
+        if (c == 0) { part[g] = M; part[G + g] = L; }
+    }
+}
+
+// One CTA per (b, row, q head); threads over channels. Splits are merged in index order.
+__global__ void attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G, int H, int D,
+                           int n_split) {
+    extern __shared__ float e[];               // [n_split] weights
+    __shared__ float red[32];
+    __shared__ float Msh;
+    const int hq = blockIdx.x % (G * H);
+    const long long br = blockIdx.x / (G * H);
+    const int h = hq / G, g = hq % G;
+    const long long stride = (long long)G * (D + 2);
+    const float* base = ws + ((br * H + h) * n_split) * stride;
+
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * stride + g]);
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = M;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float mm = -INFINITY;
+        for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) mm = fmaxf(mm, red[w]);
+        Msh = mm;
+    }
+    __syncthreads();
+    M = Msh;
+    for (int s = threadIdx.x; s < n_split; s += blockDim.x) {
+        const float ms = base[s * stride + g];
+        e[s] = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    }
+    __syncthreads();
+    float L = 0.f;
+    for (int s = 0; s < n_split; ++s) L = fmaf(base[s * stride + G + g], e[s], L);
+    const float invL = 1.f / L;
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+        float O = 0.f;
+        for (int s = 0; s < n_split; ++s) O = fmaf(base[s * stride + 2 * G + g * D + c], e[s], O);
+        out[(br * H * G + hq) * (long long)D + c] = O * invL;
+    }
+}
+
+template <int CPL>
+cudaError_t run_pass1(const P1Args& a, int n_region_split, int B, cudaStream_t st) {
+    if (n_region_split == 0) return cudaSuccess;
+    const dim3 grid(n_region_split, a.lv.H, B * a.rows);
+    const size_t smem = (size_t)P1_WARPS * a.lv.G * a.lv.D * sizeof(float);
+    attn_pass1<CPL><<<grid, 32 * P1_WARPS, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t partial_floats(int G, int D) { return (size_t)G * (D + 2); }
+
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int rows) {
+    (void)rows;
+    SplitPlan p{};
+    const long long total = n_main + n_ring;
+    const long long target = 4LL * num_sms;
+    long long per_unit = (target + units - 1) / units;
+    if (per_unit < 1) per_unit = 1;
+    long long chunk = (total + per_unit - 1) / per_unit;
+    if (chunk < 64) chunk = 64;
+    chunk = (chunk + 15) / 16 * 16;
+    p.main_chunk = p.ring_chunk = chunk;
+    p.n_main_split = (int)((n_main + chunk - 1) / chunk);
+    p.n_ring_split = (int)((n_ring + chunk - 1) / chunk);
+    return p;
+}
+
+cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, float* out,
+                             float* ws, long long n, int rows, const SplitPlan& plan,
+                             cudaStream_t st) {
+    P1Args a{};
+    a.lv = lv;
+    a.q = q;
+    a.qscale = scale * LOG2E;
+    a.ws = ws;
+    a.n = n;
+    a.pos_base = n - rows;
+    a.rows = rows;
+    a.n_split = plan.n_split();
+    const long long n_ring = lv.W ? (n < lv.W ? n : (long long)lv.W) : 0;
+    const long long n_main = n - n_ring;
+    const int CPL = lv.D / 32;
+    for (int region = 0; region < 2; ++region) {
+        a.ring = region;
+        a.chunk = region ? plan.ring_chunk : plan.main_chunk;
+        a.region_rows = region ? n_ring : n_main;
+        a.split_offset = region ? plan.n_main_split : 0;
+        const int ns = region ? plan.n_ring_split : plan.n_main_split;
+        cudaError_t e;
+        switch (CPL) {
+            case 1: e = run_pass1<1>(a, ns, lv.B, st); break;
+            case 2: e = run_pass1<2>(a, ns, lv.B, st); break;
+            case 4: e = run_pass1<4>(a, ns, lv.B, st); break;
+            case 8: e = run_pass1<8>(a, ns, lv.B, st); break;
+            default: return cudaErrorInvalidValue;
+        }
+        if (e != cudaSuccess) return e;
+    }
+    const unsigned grid = (unsigned)((long long)lv.B * rows * lv.H * lv.G);
+    const int threads = lv.D < 64 ? 64 : lv.D;
+    attn_merge<<<grid, threads, (size_t)a.n_split * sizeof(float), st>>>(ws, out, lv.G, lv.H, lv.D, a.n_split);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

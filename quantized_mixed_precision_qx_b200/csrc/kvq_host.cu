@@ -1,0 +1,296 @@
+// kvq_host.cu -- the C ABI of libkvq: cache descriptor, HBM memory map, validation,
+// split planning, launches and the canonical export.
+//
+// Everything is validated on the host before a launch; a failing call launches nothing
+// and leaves the cache length unchanged. No device memory is allocated here.
+#include "../../include/kvq.h"
+#include "kvq_internal.cuh"
+
+#include <cstring>
+#include <new>
+#include <vector>
+
+using namespace kvq;
+
+struct kvq_cache {
+    kvq_layout L;
+    int kf, vf, tf, W;
+    RowFmt fmt[2], tail;
+    // byte offsets of the areas inside the bound buffer
+    size_t off_main[2], off_ring[2], off_scales;
+    size_t main_region[2], ring_region;   // bytes per (layer, b, h) region
+    size_t total;
+    uint8_t* buf;
+    size_t buf_bytes;
+    int device, num_sms;
+    std::vector<long long> n;            // per layer
+    std::vector<char> scales_set;        // per layer (kvarn)
+};
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+LayerView layer_view(const kvq_cache* c, int layer) {
+    LayerView v{};
+    const size_t units = (size_t)c->L.batch * c->L.n_kv_heads;
+    for (int kv = 0; kv < 2; ++kv) {
+        v.main[kv] = c->buf + c->off_main[kv] + (size_t)layer * units * c->main_region[kv];
+        v.ring[kv] = c->W ? c->buf + c->off_ring[kv] + (size_t)layer * units * c->ring_region : nullptr;
+        v.fmt[kv] = c->fmt[kv];
+    }
+    v.main_region[0] = (long long)c->main_region[0];
+    v.main_region[1] = (long long)c->main_region[1];
+    v.ring_region = (long long)c->ring_region;
+    v.scales = c->L.kvarn ? reinterpret_cast<float*>(c->buf + c->off_scales) +
+                                (size_t)layer * units * 2 * c->L.head_dim
+                          : nullptr;
+    v.tail = c->tail;
+    v.B = c->L.batch;
+    v.H = c->L.n_kv_heads;
+    v.D = c->L.head_dim;
+    v.G = c->L.n_q_heads / c->L.n_kv_heads;
+    v.W = c->W;
+    v.kvarn = c->L.kvarn;
+    return v;
+}
+
+kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+    switch (s) {
+        case KVQ_OK: return "ok";
+        case KVQ_ERR_INVALID_ARG: return "invalid argument";
+        case KVQ_ERR_UNSUPPORTED_FMT: return "unsupported format";
+        case KVQ_ERR_CAPACITY: return "capacity exceeded";
+        case KVQ_ERR_CALIBRATION: return "KVarN calibration needs a longer first append";
+        case KVQ_ERR_EMPTY: return "empty cache";
+        case KVQ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case KVQ_ERR_NOT_BOUND: return "no device buffer bound";
+        case KVQ_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_fmt, kvq_fmt tail_fmt,
+                            int32_t W, kvq_cache** out) {
+    if (!layout || !out) return KVQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    const kvq_layout& L = *layout;
+    if (L.n_layers < 1 || L.batch < 1 || L.n_kv_heads < 1 || L.n_q_heads < L.n_kv_heads ||
+        L.n_q_heads % L.n_kv_heads || L.max_ctx < 1 || L.max_ctx > (1LL << 31) || L.reserved != 0)
+        return KVQ_ERR_INVALID_ARG;
+    const int D = L.head_dim;
+    if (D != 32 && D != 64 && D != 128 && D != 256) return KVQ_ERR_INVALID_ARG;
+    const int G = L.n_q_heads / L.n_kv_heads;
+    if (G > 8) return KVQ_ERR_INVALID_ARG;
+    if (L.kvarn != 0 && L.kvarn != 1) return KVQ_ERR_INVALID_ARG;
+    if (L.kvarn) {
+        const int T = L.kvarn_calib_tokens;
+        if (T < 64 || T > 1024 || (T & (T - 1)) || !(L.kvarn_eps >= 0.0)) return KVQ_ERR_INVALID_ARG;
+    }
+    if (!is_lowbit(k_fmt) || !is_lowbit(v_fmt)) return KVQ_ERR_UNSUPPORTED_FMT;
+    if (W < 0 || W > L.max_ctx) return KVQ_ERR_INVALID_ARG;
+    if (W == 0 && tail_fmt != KVQ_NONE) return KVQ_ERR_INVALID_ARG;
+    if (W > 0 && !(tail_fmt == KVQ_Q8_0 || tail_fmt == KVQ_BF16 || tail_fmt == KVQ_F16))
+        return KVQ_ERR_UNSUPPORTED_FMT;
+
+    kvq_cache* c = new (std::nothrow) kvq_cache();
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    c->L = L;
+    c->kf = k_fmt; c->vf = v_fmt; c->tf = tail_fmt; c->W = W;
+    c->fmt[0] = make_rowfmt(k_fmt, D);
+    c->fmt[1] = make_rowfmt(v_fmt, D);
+    if (W) c->tail = make_rowfmt(tail_fmt, D);
+    const size_t units = (size_t)L.n_layers * L.batch * L.n_kv_heads;
+    size_t off = 0;
+    for (int kv = 0; kv < 2; ++kv) {
+        c->main_region[kv] = align_up((size_t)L.max_ctx * c->fmt[kv].stride, 256);
+        c->off_main[kv] = off;
+        off += units * c->main_region[kv];
+    }
+    c->ring_region = W ? align_up((size_t)W * c->tail.stride, 256) : 0;
+    for (int kv = 0; kv < 2; ++kv) {
+        c->off_ring[kv] = off;
+        off += units * c->ring_region;
+    }
+    c->off_scales = off;
+    if (L.kvarn) off += align_up(units * 2 * D * sizeof(float), 256);
+    c->total = off;
+    c->buf = nullptr;
+    c->buf_bytes = 0;
+    c->device = -1;
+    c->num_sms = 0;
+    c->n.assign(L.n_layers, 0);
+    c->scales_set.assign(L.n_layers, 0);
+    *out = c;
+    return KVQ_OK;
+}
+
+kvq_status kvq_cache_required_bytes(const kvq_cache* c, size_t* bytes) {
+    if (!c || !bytes) return KVQ_ERR_INVALID_ARG;
+    *bytes = c->total;
+    return KVQ_OK;
+}
+
+kvq_status kvq_cache_bind(kvq_cache* c, void* dev_buf, size_t bytes, void* stream) {
+    if (!c || !dev_buf) return KVQ_ERR_INVALID_ARG;
+    if (((uintptr_t)dev_buf & 255) != 0) return KVQ_ERR_ALIGNMENT;
+    if (bytes < c->total) return KVQ_ERR_CAPACITY;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemsetAsync(dev_buf, 0, c->total, (cudaStream_t)stream) != cudaSuccess) return KVQ_ERR_CUDA;
+    c->buf = (uint8_t*)dev_buf;
+    c->buf_bytes = bytes;
+    c->device = dev;
+    c->num_sms = sms;
+    std::fill(c->n.begin(), c->n.end(), 0);
+    std::fill(c->scales_set.begin(), c->scales_set.end(), 0);
+    return KVQ_OK;
+}
+
+kvq_status kvq_cache_destroy(kvq_cache* c) {
+    delete c;
+    return KVQ_OK;
+}
+
+kvq_status kvq_length(const kvq_cache* c, int32_t layer, int64_t* n) {
+    if (!c || !n || layer < 0 || layer >= c->L.n_layers) return KVQ_ERR_INVALID_ARG;
+    *n = c->n[layer];
+    return KVQ_OK;
+}
+
+kvq_status kvq_set_channel_scales(kvq_cache* c, int32_t layer, const float* sK, const float* sV, void* stream) {
+    if (!c || !sK || !sV || layer < 0 || layer >= c->L.n_layers || !c->L.kvarn) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    if (!aligned16(sK) || !aligned16(sV)) return KVQ_ERR_ALIGNMENT;
+    if (c->n[layer] != 0) return KVQ_ERR_INVALID_ARG;
+    const LayerView v = layer_view(c, layer);
+    const size_t row = (size_t)c->L.head_dim * sizeof(float);
+    // device layout [B][H][2][D]: interleave K and V rows with two strided copies
+    const int BH = c->L.batch * c->L.n_kv_heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpy2DAsync(v.scales, 2 * row, sK, row, row, BH, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpy2DAsync((uint8_t*)v.scales + row, 2 * row, sV, row, row, BH, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    c->scales_set[layer] = 1;
+    return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache* c, int32_t layer, const float* k, const float* v, int32_t n_new, void* stream) {
+    if (!c || layer < 0 || layer >= c->L.n_layers || n_new < 0) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    if (n_new == 0) return KVQ_OK;
+    if (!k || !v) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGNMENT;
+    const long long n = c->n[layer];
+    if (n + n_new > c->L.max_ctx) return KVQ_ERR_CAPACITY;
+    cudaStream_t st = (cudaStream_t)stream;
+    const LayerView lv = layer_view(c, layer);
+    if (c->L.kvarn && !c->scales_set[layer]) {
+        if (n != 0 || n_new < c->L.kvarn_calib_tokens) return KVQ_ERR_CALIBRATION;
+        kvq_status s = cuda_status(launch_calibrate(lv, k, v, n_new, c->L.kvarn_calib_tokens, c->L.kvarn_eps, st));
+        if (s != KVQ_OK) return s;
+        c->scales_set[layer] = 1;
+    }
+    kvq_status s = cuda_status(launch_append(lv, k, v, n, n_new, st));
+    if (s != KVQ_OK) return s;
+    c->n[layer] = n + n_new;
+    return KVQ_OK;
+}
+
+kvq_status kvq_decode_workspace_bytes(const kvq_cache* c, int32_t n_query_rows, size_t* bytes) {
+    if (!c || !bytes || n_query_rows < 1) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    const long long units = (long long)c->L.batch * c->L.n_kv_heads * n_query_rows;
+    const long long per_unit = (4LL * c->num_sms + units - 1) / units;
+    const long long max_split = (per_unit < 1 ? 1 : per_unit) + 2;
+    const int G = c->L.n_q_heads / c->L.n_kv_heads;
+    *bytes = (size_t)units * max_split * partial_floats(G, c->L.head_dim) * sizeof(float);
+    return KVQ_OK;
+}
+
+static kvq_status attention_common(kvq_cache* c, int32_t layer, const float* q, int rows, float scale,
+                                   float* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!c || layer < 0 || layer >= c->L.n_layers || !q || !out || !ws) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(ws)) return KVQ_ERR_ALIGNMENT;
+    const long long n = c->n[layer];
+    if (n == 0) return KVQ_ERR_EMPTY;
+    if (rows < 1 || rows > n) return KVQ_ERR_INVALID_ARG;
+    size_t need = 0;
+    kvq_status s = kvq_decode_workspace_bytes(c, rows, &need);
+    if (s != KVQ_OK) return s;
+    if (ws_bytes < need) return KVQ_ERR_CAPACITY;
+    const LayerView lv = layer_view(c, layer);
+    const long long n_ring = c->W ? (n < c->W ? n : c->W) : 0;
+    const long long units = (long long)c->L.batch * c->L.n_kv_heads * rows;
+    const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, rows);
+    return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, rows, plan, (cudaStream_t)stream));
+}
+
+kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const float* q, float scale, float* out, void* ws,
+                                size_t ws_bytes, void* stream) {
+    return attention_common(c, layer, q, 1, scale, out, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, int32_t n_chunk, float scale,
+                                 float* out, void* ws, size_t ws_bytes, void* stream) {
+    if (n_chunk < 1) return KVQ_ERR_INVALID_ARG;
+    return attention_common(c, layer, q, n_chunk, scale, out, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32_t h, int32_t kv, int32_t region,
+                             int64_t pos0, int64_t count, void* host_dst, size_t bytes) {
+    if (!c || !host_dst || layer < 0 || layer >= c->L.n_layers || b < 0 || b >= c->L.batch || h < 0 ||
+        h >= c->L.n_kv_heads || kv < 0 || kv > 1 || pos0 < 0 || count < 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    const RowFmt* f;
+    const uint8_t* base;
+    const LayerView lv = layer_view(c, layer);
+    if (region == 0) {
+        if (pos0 + count > c->L.max_ctx) return KVQ_ERR_INVALID_ARG;
+        f = &c->fmt[kv];
+        base = lv.main[kv] + (size_t)(b * c->L.n_kv_heads + h) * c->main_region[kv];
+    } else if (region == 1) {
+        if (!c->W || pos0 + count > c->W) return KVQ_ERR_INVALID_ARG;
+        f = &c->tail;
+        base = lv.ring[kv] + (size_t)(b * c->L.n_kv_heads + h) * c->ring_region;
+    } else {
+        return KVQ_ERR_INVALID_ARG;
+    }
+    const int D = c->L.head_dim, nb = D / 32;
+    const size_t canon_row = (size_t)f->row_bytes;   // same bytes, block-major order
+    if (bytes < (size_t)count * canon_row) return KVQ_ERR_CAPACITY;
+    if (count == 0) return KVQ_OK;
+    std::vector<uint8_t> tmp((size_t)count * f->stride);
+    if (cudaDeviceSynchronize() != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemcpy(tmp.data(), base + (size_t)pos0 * f->stride, tmp.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    uint8_t* dst = (uint8_t*)host_dst;
+    for (int64_t r = 0; r < count; ++r) {
+        const uint8_t* row = tmp.data() + (size_t)r * f->stride;
+        uint8_t* o = dst + (size_t)r * canon_row;
+        if (f->kind != 0) {
+            std::memcpy(o, row, canon_row);
+            continue;
+        }
+        for (int blk = 0; blk < nb; ++blk) {
+            std::memcpy(o, row + 2 * blk, 2); o += 2;
+            if (f->asym) { std::memcpy(o, row + f->off_m + 2 * blk, 2); o += 2; }
+            std::memcpy(o, row + f->off_p0 + 4 * f->w0 * blk, 4 * f->w0); o += 4 * f->w0;
+            if (f->w1) { std::memcpy(o, row + f->off_p1 + 4 * f->w1 * blk, 4 * f->w1); o += 4 * f->w1; }
+        }
+    }
+    return KVQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// kvq_internal.cuh -- device-side layout, format descriptors and kernel entry points
+// shared by the libkvq translation units (CUDA path only).
+//
+// HBM layout of a bound cache (all regions 256-byte aligned):
+//   K main  [L][B][H] regions of max_ctx rows (K format row stride)
+//   V main  [L][B][H] regions of max_ctx rows (V format row stride)
+//   K ring  [L][B][H] regions of W rows (tail format row stride)        (W > 0)
+//   V ring  [L][B][H] regions of W rows                                  (W > 0)
+//   scales  [L][B][H][2][D] float32 KVarN channel scales                 (kvarn)
+// A low-bit row of D channels (nb = D/32 blocks) is stored as
+//   [d: nb x fp16][m: nb x fp16, qX_1 only][plane0: D*w0/8 bytes][plane1: D*w1/8 bytes]
+// padded to 16 bytes. Each plane is the little-endian bitstream of the row's codes in
+// channel order (channel c at bits [c*w, c*w + w)), so block b of a plane is the
+// contiguous byte range [b*4w, (b+1)*4w): the canonical per-block serialisation is a
+// byte permutation of this row. A bf16 / f16 row is D x 2 bytes.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+namespace kvq {
+
+enum : int {
+    F_Q2_0 = 0, F_Q2_1, F_Q3_0, F_Q3_1, F_Q4_0, F_Q4_1, F_Q5_0, F_Q5_1, F_Q6_0, F_Q6_1, F_Q8_0, F_Q8_1,
+    F_BF16 = 12, F_F16 = 13, F_NONE = 14
+};
+
+__host__ __device__ inline bool is_lowbit(int f) { return f >= F_Q2_0 && f <= F_Q8_1; }
+__host__ __device__ inline int fmt_bits(int f) {
+    return is_lowbit(f) ? ((f / 2 == 5) ? 8 : 2 + f / 2) : 16;
+}
+__host__ __device__ inline bool fmt_asym(int f) { return is_lowbit(f) && (f & 1); }
+
+// Runtime description of one row format (same for main-store and ring rows).
+struct RowFmt {
+    int kind;      // 0: block-quantized, 1: bf16, 2: f16
+    int bits;      // X
+    int asym;      // qX_1
+    int w0, w1;    // plane widths, low bits first (w1 = 0: one plane)
+    int off_m;     // byte offset of the mins
+    int off_p0;    // byte offset of plane 0
+    int off_p1;    // byte offset of plane 1
+    int stride;    // row stride in bytes (multiple of 16)
+    int row_bytes; // unpadded bytes of one row
+};
+
+__host__ inline RowFmt make_rowfmt(int f, int D) {
+    RowFmt r{};
+    const int nb = D / 32;
+    if (f == F_BF16 || f == F_F16) {
+        r.kind = (f == F_BF16) ? 1 : 2;
+        r.bits = 16;
+        r.row_bytes = 2 * D;
+    } else {
+        r.kind = 0;
+        r.bits = fmt_bits(f);
+        r.asym = fmt_asym(f) ? 1 : 0;
+        switch (r.bits) {
+            case 8: r.w0 = 8; r.w1 = 0; break;
+            case 6: r.w0 = 4; r.w1 = 2; break;
+            case 5: r.w0 = 4; r.w1 = 1; break;
+            case 4: r.w0 = 4; r.w1 = 0; break;
+            case 3: r.w0 = 2; r.w1 = 1; break;
+            default: r.w0 = 2; r.w1 = 0; break;
+        }
+        r.off_m = 2 * nb;
+        r.off_p0 = 2 * nb * (r.asym ? 2 : 1);
+        r.off_p1 = r.off_p0 + D * r.w0 / 8;
+        r.row_bytes = r.off_p1 + D * r.w1 / 8;
+    }
+    r.stride = (r.row_bytes + 15) & ~15;
+    return r;
+}
+
+// Per-layer view handed to kernels.
+struct LayerView {
+    uint8_t* main[2];      // K / V main area of this layer: [B][H] regions
+    uint8_t* ring[2];      // K / V ring area of this layer (nullptr if W == 0)
+    float* scales;         // [B][H][2][D] (nullptr unless kvarn)
+    long long main_region[2]; // K / V bytes per (b, h) main region
+    long long ring_region; // bytes per (b, h) ring region
+    RowFmt fmt[2];         // K / V low-bit formats
+    RowFmt tail;           // tail format (kind 0 = q8_0)
+    int B, H, D, G, W;
+    int kvarn;
+};
+
+// ---------------------------------------------------------------- launches
+cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
+                          cudaStream_t st);
+cudaError_t launch_calibrate(const LayerView& lv, const float* k, const float* v, int C, int T,
+                             double eps, cudaStream_t st);
+
+// Split plan of one attention call: every (b, h, query row) unit is cut into
+// n_main_split pieces over the low-bit rows and n_ring_split pieces over the ring.
+struct SplitPlan {
+    int n_main_split, n_ring_split;
+    long long main_chunk, ring_chunk;  // rows per split
+    int n_split() const { return n_main_split + n_ring_split; }
+};
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int rows);
+size_t partial_floats(int G, int D);   // floats of one split partial
+
+// rows = query rows per (b, h): 1 for decode, n_chunk for prefill. q/out layout
+// [B][rows][Hq][D]. pos_base: position of query row 0 (n - rows); decode uses rows = 1
+// and pos_base = n - 1 so every row sees all n positions.
+cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, float* out,
+                             float* ws, long long n, int rows, const SplitPlan& plan,
+                             cudaStream_t st);
+
+}  // namespace kvq

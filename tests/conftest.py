@@ -28,3 +28,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _build_libraries():
+    """Compile the oracle (g++) and libkvq (nvcc, sm_100a) in-tree if stale."""
+    import oracle
+    from quantized_mixed_precision_qx_b200 import build
+    oracle.build()
+    build.build()
