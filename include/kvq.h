@@ -147,6 +147,27 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const f
 KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const float* q, int32_t n_chunk,
                                  float scale, float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Decode attention exactly as kvq_decode_attention, but without a caller workspace and
+ * without allocating anything: the softmax partials go to a fixed array of
+ * KVQ_NOALLOC_WORKSPACE_MIB MiB inside the library's device image. For callers that
+ * cannot call cudaMalloc or pass a workspace (e.g. a plugin inside a host program that
+ * owns the device allocator, or a C caller whose device footprint must stay fixed after
+ * start-up). The pages have no counterpart to this entry point; it is a deployment aid.
+ *  - Every GPU that loads the library holds the array until the process exits.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with the cache's device current; make that first call before any stream capture.
+ *  - The cache's device must be the current device (KVQ_ERR_INVALID_ARG otherwise).
+ *  - A cache whose decode needs more workspace than the array holds
+ *    (kvq_decode_workspace_bytes(cache, 1) > KVQ_NOALLOC_WORKSPACE_MIB MiB) is rejected
+ *    with KVQ_ERR_CAPACITY before anything is launched.
+ *  - All calls share the array and it keeps the last call's contents (nothing in it has
+ *    to start at zero). Calls whose kernels overlap on the GPU race on it: issue them on
+ *    one stream, one after another.
+ * Calls no cudaMalloc, cudaFree or allocating routine. */
+#define KVQ_NOALLOC_WORKSPACE_MIB 8
+KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const float* q, float scale,
+                                        float* out, void* stream);
+
 /* Current number of cached positions of `layer` (host-tracked, uniform over batch). */
 KVQ_API kvq_status kvq_length(const kvq_cache* cache, int32_t layer, int64_t* n);
 

@@ -294,3 +294,62 @@ kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation.
+//
+// Some callers cannot call cudaMalloc or hand the library a workspace: for example a
+// plugin running inside a host program that owns the device allocator and gives its
+// extensions no way to reach it, or a C caller that must keep its device footprint fixed
+// once it has started. kvq_decode_attention_noalloc serves them by running the same
+// split-K decode with its softmax partials in the fixed array below instead of a
+// caller-provided workspace.
+//
+// The array lives in this library's device image: every GPU on which the library is
+// loaded holds its KVQ_NOALLOC_WS_BYTES until the process exits. In host code its name
+// only stands for the device symbol; the device address is looked up once per device
+// with cudaGetSymbolAddress (on the entry point's first call on that device, with that
+// device current) and cached. Every call shares the array and it keeps the last call's
+// contents; the decode's first pass writes every partial the merge reads, so nothing has
+// to start at zero. Calls whose kernels overlap on the GPU (several streams, several
+// threads) race on the array.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr size_t KVQ_NOALLOC_WS_BYTES = (size_t)KVQ_NOALLOC_WORKSPACE_MIB << 20;
+constexpr int KVQ_MAX_DEVICES = 64;
+static __device__ __align__(256) unsigned char g_noalloc_ws[KVQ_NOALLOC_WS_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[KVQ_MAX_DEVICES] = {};
+
+// Device address of g_noalloc_ws on `dev` (which must be current), looked up once.
+kvq_status noalloc_workspace(int dev, void** ptr) {
+    if (dev < 0 || dev >= KVQ_MAX_DEVICES) return KVQ_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) return KVQ_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return KVQ_OK;
+}
+}  // namespace
+
+extern "C" kvq_status kvq_decode_attention_noalloc(kvq_cache* c, int32_t layer, const float* q, float scale,
+                                                   float* out, void* stream) {
+    if (!c || layer < 0 || layer >= c->L.n_layers || !q || !out) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (dev != c->device) return KVQ_ERR_INVALID_ARG;
+    size_t need = 0;
+    kvq_status s = kvq_decode_workspace_bytes(c, 1, &need);
+    if (s != KVQ_OK) return s;
+    if (need > KVQ_NOALLOC_WS_BYTES) return KVQ_ERR_CAPACITY;
+    void* ws = nullptr;
+    s = noalloc_workspace(dev, &ws);
+    if (s != KVQ_OK) return s;
+    return attention_common(c, layer, q, 1, scale, out, ws, KVQ_NOALLOC_WS_BYTES, stream);
+}

@@ -25,7 +25,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_FMT, ERR_CAPACITY, ERR_CALIBRATION, ERR_EMP
 
 EXPORTED = ["kvq_cache_create", "kvq_cache_required_bytes", "kvq_cache_bind", "kvq_cache_destroy",
             "kvq_append", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_prefill_attention",
-            "kvq_length", "kvq_set_channel_scales", "kvq_export_blocks", "kvq_status_string"]
+            "kvq_length", "kvq_set_channel_scales", "kvq_export_blocks", "kvq_status_string",
+            "kvq_decode_attention_noalloc"]
+NOALLOC_WORKSPACE_BYTES = 8 << 20     # KVQ_NOALLOC_WORKSPACE_MIB
 
 
 class kvq_layout(ctypes.Structure):
@@ -61,6 +63,7 @@ def lib():
             "kvq_decode_workspace_bytes": [p, i32, ctypes.POINTER(sz)],
             "kvq_decode_attention": [p, i32, p, f32, p, p, sz, p],
             "kvq_prefill_attention": [p, i32, p, i32, f32, p, p, sz, p],
+            "kvq_decode_attention_noalloc": [p, i32, p, f32, p, p],
             "kvq_length": [p, i32, ctypes.POINTER(i64)],
             "kvq_set_channel_scales": [p, i32, p, p, p],
             "kvq_export_blocks": [p, i32, i32, i32, i32, i32, i64, i64, p, sz],
@@ -135,6 +138,12 @@ def kvq_decode_attention(cache, layer: int, q, scale: float, out, ws, ws_bytes: 
 def kvq_prefill_attention(cache, layer: int, q, n_chunk: int, scale: float, out, ws, ws_bytes: int, stream=None):
     _check(lib().kvq_prefill_attention(cache, layer, _dptr(q), n_chunk, scale, _dptr(out), _dptr(ws), ws_bytes,
                                        _stream(stream)), "kvq_prefill_attention")
+
+
+def kvq_decode_attention_noalloc(cache, layer: int, q, scale: float, out, stream=None):
+    """Decode with the library's fixed device array as workspace (no allocation)."""
+    _check(lib().kvq_decode_attention_noalloc(cache, layer, _dptr(q), scale, _dptr(out), _stream(stream)),
+           "kvq_decode_attention_noalloc")
 
 
 def kvq_length(cache, layer: int) -> int:
