@@ -12,6 +12,7 @@
 // Scores are kept in base-2 units: q is pre-multiplied by scale * log2(e), so
 // p = exp2(s - m) equals exp(scale * q.k - max).
 #include "kvq_rowio.cuh"
+#include "kvq_tc_launch.cuh"
 
 #include <cfloat>
 
@@ -165,42 +166,73 @@ attn_pass1(P1Args a) {
     }
 }
 
-// One CTA per (b, row, q head); threads over channels. Splits are merged in index order.
-__global__ void attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G, int H, int D,
-                           int n_split) {
+// Merge of the split partials. One CTA per (b, row, q head) and 32-channel slice; its
+// 256 threads are 32 channels x 8 split groups. Weights e_s = 2^(m_s - M) go to shared
+// memory; group j sums splits j, j+8, j+16, ... in order and the 8 group sums are added
+// in a fixed order, so the result is bit-reproducible.
+constexpr int MG = 8;
+__global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G,
+                                                  int H, int D, int n_split) {
     extern __shared__ float e[];               // [n_split] weights
-    __shared__ float red[32];
-    __shared__ float Msh;
+    __shared__ float red[MG][32];
+    __shared__ float wred[8];
+    __shared__ float Msh, Lsh;
     const int hq = blockIdx.x % (G * H);
     const long long br = blockIdx.x / (G * H);
     const int h = hq / G, g = hq % G;
     const long long stride = (long long)G * (D + 2);
     const float* base = ws + ((br * H + h) * n_split) * stride;
+    const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
 
     float M = -INFINITY;
-    for (int s = threadIdx.x; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * stride + g]);
+    for (int s = tid; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * stride + g]);
     for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = M;
+    if (lane == 0) wred[grp] = M;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         float mm = -INFINITY;
-        for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) mm = fmaxf(mm, red[w]);
+        for (int w = 0; w < MG; ++w) mm = fmaxf(mm, wred[w]);
         Msh = mm;
     }
     __syncthreads();
     M = Msh;
-    for (int s = threadIdx.x; s < n_split; s += blockDim.x) {
+    float lpart = 0.f;                         // fixed assignment: thread tid sums splits tid, tid+256, ...
+    for (int s = tid; s < n_split; s += blockDim.x) {
         const float ms = base[s * stride + g];
-        e[s] = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        e[s] = w;
+        lpart = fmaf(base[s * stride + G + g], w, lpart);
     }
+    for (int off = 16; off >= 1; off >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, off);
     __syncthreads();
-    float L = 0.f;
-    for (int s = 0; s < n_split; ++s) L = fmaf(base[s * stride + G + g], e[s], L);
-    const float invL = 1.f / L;
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    if (lane == 0) wred[grp] = lpart;
+    __syncthreads();
+    if (tid == 0) {
+        float L = 0.f;
+        for (int w = 0; w < MG; ++w) L += wred[w];
+        Lsh = L;
+    }
+    const int c = blockIdx.y * 32 + lane;
+    float acc = 0.f;
+    if (c < D) {
+        const float* ob = base + 2 * G + (long long)g * D + c;
+        int s = grp;
+        for (; s + 3 * MG < n_split; s += 4 * MG) {
+            const float o0 = ob[(long long)s * stride], o1 = ob[(long long)(s + MG) * stride];
+            const float o2 = ob[(long long)(s + 2 * MG) * stride], o3 = ob[(long long)(s + 3 * MG) * stride];
+            acc = fmaf(o0, e[s], acc);
+            acc = fmaf(o1, e[s + MG], acc);
+            acc = fmaf(o2, e[s + 2 * MG], acc);
+            acc = fmaf(o3, e[s + 3 * MG], acc);
+        }
+        for (; s < n_split; s += MG) acc = fmaf(ob[(long long)s * stride], e[s], acc);
+    }
+    red[grp][lane] = acc;
+    __syncthreads();
+    if (grp == 0 && c < D) {
         float O = 0.f;
-        for (int s = 0; s < n_split; ++s) O = fmaf(base[s * stride + 2 * G + g * D + c], e[s], O);
-        out[(br * H * G + hq) * (long long)D + c] = O * invL;
+        for (int j = 0; j < MG; ++j) O += red[j][lane];
+        out[(br * H * G + hq) * (long long)D + c] = O / Lsh;
     }
 }
 
@@ -217,19 +249,27 @@ cudaError_t run_pass1(const P1Args& a, int n_region_split, int B, cudaStream_t s
 
 size_t partial_floats(int G, int D) { return (size_t)G * (D + 2); }
 
-SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int rows) {
-    (void)rows;
+bool use_tensor_cores(int D) { return D == 128 || D == 256; }
+
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, bool tc) {
     SplitPlan p{};
     const long long total = n_main + n_ring;
-    const long long target = 4LL * num_sms;
+    const long long target = (tc ? 3LL : 4LL) * num_sms;
     long long per_unit = (target + units - 1) / units;
     if (per_unit < 1) per_unit = 1;
-    long long chunk = (total + per_unit - 1) / per_unit;
-    if (chunk < 64) chunk = 64;
-    chunk = (chunk + 15) / 16 * 16;
-    p.main_chunk = p.ring_chunk = chunk;
+    const long long align = tc ? tc::TOK : 16;
+    // low-bit rows: about per_unit splits of at least 4 tiles each
+    long long chunk = (n_main + per_unit - 1) / per_unit;
+    if (chunk < 4 * align) chunk = 4 * align;
+    chunk = (chunk + align - 1) / align * align;
+    // ring rows run as a separate, later launch: cut them finer so it ends quickly
+    long long rchunk = (n_ring + per_unit - 1) / per_unit;
+    if (rchunk < align) rchunk = align;
+    rchunk = (rchunk + align - 1) / align * align;
+    p.main_chunk = chunk;
+    p.ring_chunk = rchunk;
     p.n_main_split = (int)((n_main + chunk - 1) / chunk);
-    p.n_ring_split = (int)((n_ring + chunk - 1) / chunk);
+    p.n_ring_split = (int)((n_ring + rchunk - 1) / rchunk);
     return p;
 }
 
@@ -248,25 +288,56 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     const long long n_ring = lv.W ? (n < lv.W ? n : (long long)lv.W) : 0;
     const long long n_main = n - n_ring;
     const int CPL = lv.D / 32;
+    const bool tcp = use_tensor_cores(lv.D);
     for (int region = 0; region < 2; ++region) {
         a.ring = region;
         a.chunk = region ? plan.ring_chunk : plan.main_chunk;
         a.region_rows = region ? n_ring : n_main;
         a.split_offset = region ? plan.n_main_split : 0;
         const int ns = region ? plan.n_ring_split : plan.n_main_split;
+        if (ns == 0) continue;
         cudaError_t e;
-        switch (CPL) {
-            case 1: e = run_pass1<1>(a, ns, lv.B, st); break;
-            case 2: e = run_pass1<2>(a, ns, lv.B, st); break;
-            case 4: e = run_pass1<4>(a, ns, lv.B, st); break;
-            case 8: e = run_pass1<8>(a, ns, lv.B, st); break;
-            default: return cudaErrorInvalidValue;
+        if (tcp) {
+            tc::Args t{};
+            const RowFmt& fk = region ? lv.tail : lv.fmt[0];
+            const RowFmt& fv = region ? lv.tail : lv.fmt[1];
+            t.kbase = region ? lv.ring[0] : lv.main[0];
+            t.vbase = region ? lv.ring[1] : lv.main[1];
+            t.kstride = fk.stride;
+            t.vstride = fv.stride;
+            t.q = q;
+            t.qscale = a.qscale;
+            t.scales = lv.kvarn ? lv.scales : nullptr;
+            t.ws = ws;
+            t.n = n;
+            t.pos_base = a.pos_base;
+            t.rows = rows;
+            t.ring = region;
+            t.W = lv.W;
+            t.chunk = a.chunk;
+            t.region_rows = a.region_rows;
+            t.region_stride_k = region ? lv.ring_region : lv.main_region[0];
+            t.region_stride_v = region ? lv.ring_region : lv.main_region[1];
+            t.split_offset = a.split_offset;
+            t.n_split = a.n_split;
+            t.H = lv.H;
+            t.G = lv.G;
+            t.D = lv.D;
+            const dim3 grid(ns, lv.H, lv.B * rows);
+            e = tc::launch_tc(fk.id, fv.id, t, grid, tc::smem_bytes(fk.stride, fv.stride, lv.D), st);
+        } else {
+            switch (CPL) {
+                case 1: e = run_pass1<1>(a, ns, lv.B, st); break;
+                case 2: e = run_pass1<2>(a, ns, lv.B, st); break;
+                case 4: e = run_pass1<4>(a, ns, lv.B, st); break;
+                case 8: e = run_pass1<8>(a, ns, lv.B, st); break;
+                default: return cudaErrorInvalidValue;
+            }
         }
         if (e != cudaSuccess) return e;
     }
-    const unsigned grid = (unsigned)((long long)lv.B * rows * lv.H * lv.G);
-    const int threads = lv.D < 64 ? 64 : lv.D;
-    attn_merge<<<grid, threads, (size_t)a.n_split * sizeof(float), st>>>(ws, out, lv.G, lv.H, lv.D, a.n_split);
+    const dim3 grid((unsigned)((long long)lv.B * rows * lv.H * lv.G), (unsigned)((lv.D + 31) / 32));
+    attn_merge<<<grid, 256, (size_t)a.n_split * sizeof(float), st>>>(ws, out, lv.G, lv.H, lv.D, a.n_split);
     return cudaGetLastError();
 }
 

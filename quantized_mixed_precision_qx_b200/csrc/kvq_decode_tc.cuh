@@ -1,0 +1,426 @@
+// kvq_decode_tc.cuh -- split-K decode / row-batched prefill pass 1 on warp-level tensor
+// cores, for head_dim 128 or 256 (nb = 4 or 8 blocks of 32 channels).
+//
+// CTA = 4 consumer warps + 1 producer warp. The producer streams the split's rows in
+// 64-row tiles with 1-D bulk copies (TMA engine) into a 3-stage shared-memory ring
+// (K tile and V tile are each one contiguous copy, since a region stores its rows back
+// to back). Each consumer warp takes 16 rows of every tile:
+//   S^T[16 x 8] = K[16 x D] Q^T[D x 8]   (m16n8k16; rows = tokens, 8 = the G <= 8 heads)
+//   p = exp2(S - m) with a per-head running max m and sum l (online softmax)
+//   O^T[D x 8] += V^T[D x 16] P^T[16 x 8]
+// Codes enter the MMAs exactly (fp16 integers); block scales are applied to the QK
+// accumulators per 32-channel block and folded into P for PV; the query and P*d are
+// split into hi + lo fp16 parts. At the end the 4 warps' states are merged in shared
+// memory and the CTA writes one (m, l, o) partial per head, like the CUDA-core path.
+#pragma once
+#include "kvq_mma.cuh"
+
+namespace kvq {
+namespace tc {
+
+constexpr int TOK = 64;         // rows per stage
+constexpr int STAGES = 2;
+constexpr int CWARPS = 4;       // consumer warps
+constexpr int THREADS = 32 * (CWARPS + 1);
+constexpr int NBMAX = 8;
+// Lazy rescale: a head's running max is only raised when a score exceeds it by more
+// than 2^8, so p stays <= 256 and the accumulators are rescaled rarely. Results are
+// mathematically unchanged (m, l and o always refer to the same stale max).
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+struct Args {
+    const uint8_t* kbase;   // first row of this (b, h) K region
+    const uint8_t* vbase;
+    int kstride, vstride;   // row strides (bytes)
+    const float* q;         // [B][rows][Hq][D]
+    float qscale;           // scale * log2(e)
+    const float* scales;    // KVarN [B][H][2][D] or nullptr
+    float* ws;
+    long long n;            // cached positions
+    long long pos_base;     // position of query row 0
+    int rows;
+    int ring;               // region: 0 low-bit, 1 ring
+    int W;
+    long long chunk;        // rows per split
+    long long region_rows;
+    long long region_stride_k, region_stride_v;   // bytes between (b, h) regions
+    int split_offset, n_split;
+    int H, G, D;
+};
+
+__host__ __device__ constexpr size_t stage_bytes(int ks, int vs) { return (size_t)TOK * (ks + vs); }
+// shared memory: [stages | final combine (aliased)] [P transpose] [mbarriers] [fault word]
+__host__ __device__ constexpr size_t comb_bytes(int D) {
+    return (size_t)(CWARPS * 8 * 2 + CWARPS * 8 * NBMAX + CWARPS * 8 * D) * sizeof(float);
+}
+__host__ __device__ constexpr size_t main_bytes(int ks, int vs, int D) {
+    return ((STAGES * stage_bytes(ks, vs) > comb_bytes(D) ? STAGES * stage_bytes(ks, vs) : comb_bytes(D)) + 127) & ~(size_t)127;
+}
+constexpr size_t PT_BYTES = CWARPS * 16 * 8 * sizeof(float);
+constexpr size_t QS_BYTES = NBMAX * 2 * 3 * 32 * sizeof(uint2);     // query fragments (<= 3 parts)
+constexpr size_t QSUM_BYTES = NBMAX * 8 * sizeof(float);
+__host__ __device__ constexpr size_t smem_bytes(int ks, int vs, int D) {
+    return main_bytes(ks, vs, D) + PT_BYTES + QS_BYTES + QSUM_BYTES + 2 * STAGES * sizeof(uint64_t) + 16;
+}
+
+template <int KF, int VF, int NB>
+__global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
+    using namespace mma;
+    using KT = Fmt<KF>;
+    using VT = Fmt<VF>;
+    static_assert(KT::is_bf16 == VT::is_bf16, "K and V must use the same MMA operand type");
+    constexpr int KP = KT::parts;            // parts of the query split
+    constexpr int VP = VT::parts;            // parts of the P split
+    constexpr bool VSCALED = !VT::is_float;  // block scale folded into the V operand
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int D = 32 * NB, G = a.G, H = a.H;
+    const size_t sb = stage_bytes(a.kstride, a.vstride);
+    const size_t mb = main_bytes(a.kstride, a.vstride, D);
+    uint8_t* stage0 = smem;
+    float* pT = reinterpret_cast<float*>(smem + mb);                                   // [CWARPS][16][8]
+    uint2* qs = reinterpret_cast<uint2*>(smem + mb + PT_BYTES);                        // [NB][2][KP][32]
+    float* qsum_s = reinterpret_cast<float*>(smem + mb + PT_BYTES + QS_BYTES);         // [NB][8]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + QS_BYTES + QSUM_BYTES);
+    uint64_t* empty = full + STAGES;
+    int* fault = reinterpret_cast<int*>(empty + STAGES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int h = blockIdx.y, br = blockIdx.z;
+    const int b = br / a.rows, r = br % a.rows;
+    const int split = blockIdx.x;
+    const long long limit = a.pos_base + r;
+
+    long long t0 = (long long)split * a.chunk;
+    long long t1 = t0 + a.chunk;
+    if (t1 > a.region_rows) t1 = a.region_rows;
+    if (!a.ring && t1 > limit + 1) t1 = limit + 1;
+    if (t1 < t0) t1 = t0;
+    const int n_tiles = (int)((t1 - t0 + TOK - 1) / TOK);
+
+    const uint8_t* kreg = a.kbase + (long long)(b * H + h) * a.region_stride_k;
+    const uint8_t* vreg = a.vbase + (long long)(b * H + h) * a.region_stride_v;
+    const int kvarn = a.scales != nullptr && !a.ring;
+    const float* sK = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 0) * D : nullptr;
+    const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], CWARPS); }
+        *fault = 0;
+        fence_mbar_init();
+    }
+    // Rows past the end of a partial tile are read (and multiplied by p = 0): zero the
+    // stages once so such rows always hold finite values (stale rows of this region or 0).
+    for (size_t i = threadIdx.x * 16; i < STAGES * sb; i += THREADS * 16)
+        *reinterpret_cast<uint4*>(stage0 + i) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    // query fragments (B operand of QK, head g of lane (g, t)), shared by the consumer warps
+    if (warp == 0) {
+        const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                float v[4];
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const int c = 32 * bb + q_channel<KF>(t, m, sl);
+                    float x = (g < G) ? qg[c] * a.qscale : 0.f;
+                    if (kvarn) x *= sK[c];
+                    v[sl] = x;
+                }
+                uint32_t p01[3], p23[3];
+                split_pack<KF>(v[0], v[1], p01);
+                split_pack<KF>(v[2], v[3], p23);
+#pragma unroll
+                for (int pp = 0; pp < KP; ++pp) qs[((bb * 2 + m) * KP + pp) * 32 + lane] = make_uint2(p01[pp], p23[pp]);
+            }
+        }
+        if constexpr (KT::asym) {
+            // per-block sums of the (scaled) query channels, heads 0..7
+            for (int idx = lane; idx < NB * 8; idx += 32) {
+                const int bb = idx >> 3, hh = idx & 7;
+                float sacc = 0.f;
+                if (hh < G) {
+                    const float* qh = a.q + ((long long)br * G * H + (long long)h * G + hh) * D + 32 * bb;
+                    for (int c = 0; c < 32; ++c) {
+                        float x = qh[c] * a.qscale;
+                        if (kvarn) x *= sK[32 * bb + c];
+                        sacc += x;
+                    }
+                }
+                qsum_s[idx] = sacc;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ producer warp
+    if (warp == CWARPS) {
+        if (lane == 0) {
+            for (int it = 0; it < n_tiles; ++it) {
+                const int s = it % STAGES;
+                if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) { *fault = 1; break; }
+                const long long r0 = t0 + (long long)it * TOK;
+                const int nrows = (int)min((long long)TOK, t1 - r0);
+                const uint32_t kb = (uint32_t)(nrows * a.kstride), vb = (uint32_t)(nrows * a.vstride);
+                uint8_t* st = stage0 + s * sb;
+                mbar_arrive_expect_tx(&full[s], kb + vb);
+                bulk_g2s(st, kreg + r0 * a.kstride, kb, &full[s]);
+                bulk_g2s(st + (size_t)TOK * a.kstride, vreg + r0 * a.vstride, vb, &full[s]);
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ consumers
+    float o[NB][2][4];
+    float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+    float pm[NB];                         // asym V: sum_t p_t m_t,b for head g
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb) {
+        pm[bb] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[bb][m][i] = 0.f;
+    }
+
+    if (warp < CWARPS) {
+        float* myT = pT + warp * 128;
+        const long long W = a.W;
+        const long long ring_base = a.n - W;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int s = it % STAGES;
+            if (!mbar_wait(&full[s], (it / STAGES) & 1)) { *fault = 1; break; }
+            const long long r0 = t0 + (long long)it * TOK;
+            const int nrows = (int)min((long long)TOK, t1 - r0);
+            const int sub0 = 16 * warp;
+            if (sub0 < nrows) {
+                const uint8_t* kt = stage0 + s * sb;
+                const uint8_t* vt = kt + (size_t)TOK * a.kstride;
+                auto valid = [&](int rr) -> bool {
+                    if (sub0 + rr >= nrows) return false;
+                    if (a.ring) {
+                        const long long slot = r0 + sub0 + rr;
+                        const long long pos = ring_base + ((slot - ring_base) % W + W) % W;
+                        return pos <= limit;
+                    }
+                    return true;
+                };
+                // ---------------- S^T = K Q^T
+                const uint8_t* rg = kt + (size_t)(sub0 + g) * a.kstride;
+                const uint8_t* rg8 = kt + (size_t)(sub0 + g + 8) * a.kstride;
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) {
+                    uint32_t af[2][4];
+                    k_frags<KF>(rg, rg8, NB, bb, t, af);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int pp = 0; pp < KP; ++pp) {
+                            const uint2 qv = qs[((bb * 2 + m) * KP + pp) * 32 + lane];
+                            mma_f<KF>(acc, af[m], qv.x, qv.y);
+                        }
+                    if constexpr (KT::is_float) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) sc[i] += acc[i];
+                    } else {
+                        const float dg = h2f_lo(reinterpret_cast<const uint16_t*>(rg)[bb]);
+                        const float dg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8)[bb]);
+                        sc[0] = fmaf(acc[0], dg, sc[0]);
+                        sc[1] = fmaf(acc[1], dg, sc[1]);
+                        sc[2] = fmaf(acc[2], dg8, sc[2]);
+                        sc[3] = fmaf(acc[3], dg8, sc[3]);
+                        if constexpr (KT::asym) {
+                            const float mg = h2f_lo(reinterpret_cast<const uint16_t*>(rg + KT::off_m(NB))[bb]);
+                            const float mg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8 + KT::off_m(NB))[bb]);
+                            const float2 qq = *reinterpret_cast<const float2*>(&qsum_s[bb * 8 + 2 * t]);
+                            sc[0] = fmaf(mg, qq.x, sc[0]);
+                            sc[1] = fmaf(mg, qq.y, sc[1]);
+                            sc[2] = fmaf(mg8, qq.x, sc[2]);
+                            sc[3] = fmaf(mg8, qq.y, sc[3]);
+                        }
+                    }
+                }
+                if (!valid(g)) { sc[0] = -INFINITY; sc[1] = -INFINITY; }
+                if (!valid(g + 8)) { sc[2] = -INFINITY; sc[3] = -INFINITY; }
+                // ---------------- online softmax for heads 2t, 2t+1
+                float mx0 = fmaxf(sc[0], sc[2]), mx1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const bool up0 = mx0 > mrun[0] + RESCALE_THRESHOLD || (mrun[0] == -INFINITY && mx0 > -INFINITY);
+                const bool up1 = mx1 > mrun[1] + RESCALE_THRESHOLD || (mrun[1] == -INFINITY && mx1 > -INFINITY);
+                if (__any_sync(0xffffffffu, up0 || up1)) {
+                    const float mn0 = up0 ? mx0 : mrun[0];
+                    const float mn1 = up1 ? mx1 : mrun[1];
+                    const float c0 = (mrun[0] == -INFINITY) ? 0.f : ex2(mrun[0] - mn0);
+                    const float c1 = (mrun[1] == -INFINITY) ? 0.f : ex2(mrun[1] - mn1);
+                    lrun[0] *= c0;
+                    lrun[1] *= c1;
+#pragma unroll
+                    for (int bb = 0; bb < NB; ++bb)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            o[bb][m][0] *= c0; o[bb][m][1] *= c1;
+                            o[bb][m][2] *= c0; o[bb][m][3] *= c1;
+                        }
+                    if constexpr (VT::asym) {
+                        // pm belongs to head g: fetch that head's factor from lane (g >> 1)
+                        const float f0 = __shfl_sync(0xffffffffu, c0, g >> 1);
+                        const float f1 = __shfl_sync(0xffffffffu, c1, g >> 1);
+                        const float cg = (g & 1) ? f1 : f0;
+#pragma unroll
+                        for (int bb = 0; bb < NB; ++bb) pm[bb] *= cg;
+                    }
+                    mrun[0] = mn0;
+                    mrun[1] = mn1;
+                }
+                float p[4];
+                if (mrun[0] == -INFINITY) { p[0] = 0.f; p[2] = 0.f; }
+                else { p[0] = ex2(sc[0] - mrun[0]); p[2] = ex2(sc[2] - mrun[0]); }
+                if (mrun[1] == -INFINITY) { p[1] = 0.f; p[3] = 0.f; }
+                else { p[1] = ex2(sc[1] - mrun[1]); p[3] = ex2(sc[3] - mrun[1]); }
+                lrun[0] += p[0] + p[2];
+                lrun[1] += p[1] + p[3];
+                // ---------------- transpose P: (tokens g, g+8; heads 2t, 2t+1) -> (tokens 2t.., head g)
+                *reinterpret_cast<float2*>(&myT[g * 8 + 2 * t]) = make_float2(p[0], p[1]);
+                *reinterpret_cast<float2*>(&myT[(g + 8) * 8 + 2 * t]) = make_float2(p[2], p[3]);
+                __syncwarp();
+                const int tk0 = 2 * t, tk2 = 2 * t + 8;
+                float pv[4];
+                pv[0] = myT[tk0 * 8 + g];
+                pv[1] = myT[(tk0 + 1) * 8 + g];
+                pv[2] = myT[tk2 * 8 + g];
+                pv[3] = myT[(tk2 + 1) * 8 + g];
+                __syncwarp();
+                const bool v0 = valid(tk0), v1 = valid(tk0 + 1), v2 = valid(tk2), v3 = valid(tk2 + 1);
+                const uint8_t* vr0 = vt + (size_t)(sub0 + tk0) * a.vstride;
+                const uint8_t* vr1 = vr0 + a.vstride;
+                const uint8_t* vr2 = vt + (size_t)(sub0 + tk2) * a.vstride;
+                const uint8_t* vr3 = vr2 + a.vstride;
+                // P split once per sub-tile (invalid tokens carry p = 0)
+                uint32_t bp[3][2];
+                {
+                    uint32_t x01[3], x23[3];
+                    split_pack<VF>(v0 ? pv[0] : 0.f, v1 ? pv[1] : 0.f, x01);
+                    split_pack<VF>(v2 ? pv[2] : 0.f, v3 ? pv[3] : 0.f, x23);
+#pragma unroll
+                    for (int pp = 0; pp < 3; ++pp) { bp[pp][0] = x01[pp]; bp[pp][1] = x23[pp]; }
+                }
+                // ---------------- O^T += V^T P^T
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) {
+                    if constexpr (VSCALED) {
+                        uint32_t ah[2][4], al[2][4];
+                        v_frags_scaled<VF>(vr0, vr1, vr2, vr3, NB, bb, g, ah, al);
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            mma_f16(o[bb][m], ah[m], bp[0][0], bp[0][1]);
+                            mma_f16(o[bb][m], ah[m], bp[1][0], bp[1][1]);
+                            mma_f16(o[bb][m], al[m], bp[0][0], bp[0][1]);
+                        }
+                        if constexpr (VT::asym) {
+                            const float m0 = h2f_lo(reinterpret_cast<const uint16_t*>(vr0 + VT::off_m(NB))[bb]);
+                            const float m1 = h2f_lo(reinterpret_cast<const uint16_t*>(vr1 + VT::off_m(NB))[bb]);
+                            const float m2 = h2f_lo(reinterpret_cast<const uint16_t*>(vr2 + VT::off_m(NB))[bb]);
+                            const float m3 = h2f_lo(reinterpret_cast<const uint16_t*>(vr3 + VT::off_m(NB))[bb]);
+                            float acc = pm[bb];
+                            if (v0) acc = fmaf(pv[0], m0, acc);
+                            if (v1) acc = fmaf(pv[1], m1, acc);
+                            if (v2) acc = fmaf(pv[2], m2, acc);
+                            if (v3) acc = fmaf(pv[3], m3, acc);
+                            pm[bb] = acc;
+                        }
+                    } else {
+                        uint32_t af[2][4];
+                        v_frags<VF>(vr0, vr1, vr2, vr3, NB, bb, g, af);
+#pragma unroll
+                        for (int m = 0; m < 2; ++m)
+#pragma unroll
+                            for (int pp = 0; pp < VP; ++pp) mma_f<VF>(o[bb][m], af[m], bp[pp][0], bp[pp][1]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+
+    // ------------------------------------------------------------ combine the 4 warps
+    __syncthreads();
+    // shared layout (reusing the stages): cm[CWARPS][8], cl[CWARPS][8], cpm[CWARPS][8][NBMAX], co[CWARPS][8][D]
+    float* cm = reinterpret_cast<float*>(smem);
+    float* cl = cm + CWARPS * 8;
+    float* cpm = cl + CWARPS * 8;
+    float* co = cpm + CWARPS * 8 * NBMAX;
+    if (warp < CWARPS) {
+        // l: reduce the per-thread partial sums over the 8 lanes sharing t
+        float l0 = lrun[0], l1 = lrun[1];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        }
+        if (g == 0) {
+            cm[warp * 8 + 2 * t] = mrun[0];
+            cm[warp * 8 + 2 * t + 1] = mrun[1];
+            cl[warp * 8 + 2 * t] = l0;
+            cl[warp * 8 + 2 * t + 1] = l1;
+        }
+        if constexpr (VT::asym) {
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+                float v = pm[bb];
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                if (t == 0) cpm[(warp * 8 + g) * NBMAX + bb] = v;
+            }
+        }
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int c_lo = 32 * bb + v_channel(g, m, 0), c_hi = 32 * bb + v_channel(g, m, 1);
+                co[(warp * 8 + 2 * t) * D + c_lo] = o[bb][m][0];
+                co[(warp * 8 + 2 * t + 1) * D + c_lo] = o[bb][m][1];
+                co[(warp * 8 + 2 * t) * D + c_hi] = o[bb][m][2];
+                co[(warp * 8 + 2 * t + 1) * D + c_hi] = o[bb][m][3];
+            }
+        }
+    }
+    __syncthreads();
+    float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
+    const bool bad = *fault != 0;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int hh = idx / D, c = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, cm[w * 8 + hh]);
+        float O = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < CWARPS; ++w) {
+                const float mw = cm[w * 8 + hh];
+                if (mw == -INFINITY) continue;
+                const float e = ex2(mw - M);
+                float ow = co[(w * 8 + hh) * D + c];
+                if constexpr (VT::asym) ow += cpm[(w * 8 + hh) * NBMAX + (c >> 5)];
+                O = fmaf(ow, e, O);
+                L = fmaf(cl[w * 8 + hh], e, L);
+            }
+        }
+        if (sV) O *= sV[c];
+        if (bad) L = __int_as_float(0x7fc00000);   // a timed-out wait poisons the result
+        part[2 * G + idx] = O;
+        if (c == 0) { part[hh] = M; part[G + hh] = L; }
+    }
+}
+
+}  // namespace tc
+}  // namespace kvq

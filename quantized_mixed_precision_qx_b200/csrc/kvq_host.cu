@@ -210,8 +210,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache* c, int32_t n_query_rows, 
     if (!c || !bytes || n_query_rows < 1) return KVQ_ERR_INVALID_ARG;
     if (!c->buf) return KVQ_ERR_NOT_BOUND;
     const long long units = (long long)c->L.batch * c->L.n_kv_heads * n_query_rows;
+    // main and ring splits are each at most per_unit + 1 (see plan_splits)
     const long long per_unit = (4LL * c->num_sms + units - 1) / units;
-    const long long max_split = (per_unit < 1 ? 1 : per_unit) + 2;
+    const long long max_split = 2 * (per_unit < 1 ? 1 : per_unit) + 2;
     const int G = c->L.n_q_heads / c->L.n_kv_heads;
     *bytes = (size_t)units * max_split * partial_floats(G, c->L.head_dim) * sizeof(float);
     return KVQ_OK;
@@ -232,7 +233,7 @@ static kvq_status attention_common(kvq_cache* c, int32_t layer, const float* q, 
     const LayerView lv = layer_view(c, layer);
     const long long n_ring = c->W ? (n < c->W ? n : c->W) : 0;
     const long long units = (long long)c->L.batch * c->L.n_kv_heads * rows;
-    const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, rows);
+    const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, use_tensor_cores(c->L.head_dim));
     return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, rows, plan, (cudaStream_t)stream));
 }
 

@@ -34,6 +34,7 @@ __host__ __device__ inline bool fmt_asym(int f) { return is_lowbit(f) && (f & 1)
 
 // Runtime description of one row format (same for main-store and ring rows).
 struct RowFmt {
+    int id;        // kvq_fmt value
     int kind;      // 0: block-quantized, 1: bf16, 2: f16
     int bits;      // X
     int asym;      // qX_1
@@ -47,6 +48,7 @@ struct RowFmt {
 
 __host__ inline RowFmt make_rowfmt(int f, int D) {
     RowFmt r{};
+    r.id = f;
     const int nb = D / 32;
     if (f == F_BF16 || f == F_F16) {
         r.kind = (f == F_BF16) ? 1 : 2;
@@ -99,7 +101,9 @@ struct SplitPlan {
     long long main_chunk, ring_chunk;  // rows per split
     int n_split() const { return n_main_split + n_ring_split; }
 };
-SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int rows);
+// Tensor-core path (head_dim 128 / 256) when tc is set: splits are whole 64-row tiles.
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, bool tc);
+bool use_tensor_cores(int D);
 size_t partial_floats(int G, int D);   // floats of one split partial
 
 // rows = query rows per (b, h): 1 for decode, n_chunk for prefill. q/out layout

@@ -1,0 +1,396 @@
+// kvq_mma.cuh -- register-level building blocks of the tensor-core decode kernel:
+// m16n8k16 MMAs, TMA bulk copies with mbarriers (bounded waits), and the per-format
+// unpacking of packed code planes straight into MMA A-fragments.
+//
+// Exactness: a qX code (offset removed) is a small integer and exact in fp16, so the
+// A operand carries codes without rounding. The other operand (the query, or the
+// softmax weight times the block scale) is split into fp16 hi + lo parts, so each
+// product is carried to ~22 significant bits with fp32 accumulation. A 16-bit float
+// ring row is exact in its own type; bf16 rows pair with a 3-way bf16 split.
+#pragma once
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace mma {
+
+// ---------------------------------------------------------------- formats
+template <int F>
+struct Fmt {
+    static constexpr bool is_float = (F == F_BF16 || F == F_F16);
+    static constexpr bool is_bf16 = (F == F_BF16);
+    static constexpr int bits = is_float ? 16 : ((F / 2 == 5) ? 8 : 2 + F / 2);
+    static constexpr bool asym = !is_float && (F & 1);
+    static constexpr int w0 = is_float ? 16 : (bits == 8 ? 8 : (bits >= 4 ? 4 : 2));
+    static constexpr int w1 = is_float ? 0 : bits - w0;
+    static constexpr int off = asym ? 0 : (is_float ? 0 : (1 << (bits - 1)));
+    // row byte offsets for nb blocks (see kvq_internal.cuh)
+    __device__ static constexpr int off_m(int nb) { return 2 * nb; }
+    __device__ static constexpr int off_p0(int nb) { return is_float ? 0 : 2 * nb * (asym ? 2 : 1); }
+    __device__ static constexpr int off_p1(int nb) { return off_p0(nb) + 32 * nb * w0 / 8; }
+    // number of B-operand parts (split of the non-code operand)
+    static constexpr int parts = is_bf16 ? 3 : 2;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// (a & mask) | c  in one LOP3
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t c) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(c));
+    return r;
+}
+
+template <int S>
+__device__ __forceinline__ uint32_t shift(uint32_t x) {   // S > 0: left, S < 0: right
+    if constexpr (S > 0) return x << S;
+    else if constexpr (S < 0) return x >> (-S);
+    else return x;
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int F>
+__device__ __forceinline__ void mma_f(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (Fmt<F>::is_bf16) mma_bf16(c, a, b0, b1);
+    else mma_f16(c, a, b0, b1);
+}
+
+// Exact fp16 -> fp32 without the conversion unit: the fp16 bit pattern shifted into the
+// fp32 exponent/mantissa fields is the fp32 value x * 2^-112 (normal or subnormal fp16
+// alike), so one exact multiply by 2^112 restores x. lo16 / hi16 select a half of w.
+__device__ __forceinline__ float h2f_lo(uint32_t w) {
+    const uint32_t u = ((w << 13) & 0x0FFFE000u) | ((w << 16) & 0x80000000u);
+    return __uint_as_float(u) * 5.192296858534828e33f;   // 2^112
+}
+__device__ __forceinline__ float h2f_hi(uint32_t w) {
+    const uint32_t u = ((w >> 3) & 0x0FFFE000u) | (w & 0x80000000u);
+    return __uint_as_float(u) * 5.192296858534828e33f;
+}
+
+// 2^x on the special-function unit (relative error ~2^-22; inputs <= 0 or small)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Split x into `parts` values of the MMA's 16-bit type whose sum carries x to about
+// 11 (fp16) or 8 (bf16) significant bits per part. The high part is x with its fp32
+// mantissa truncated to the 16-bit type's width (exactly representable in range), the
+// next part is the exact fp32 remainder, rounded; two values pack into one register.
+template <int F>
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t (&out)[3]) {
+    if constexpr (Fmt<F>::is_bf16) {
+        const float h0 = __uint_as_float(__float_as_uint(x0) & 0xFFFF0000u);
+        const float h1 = __uint_as_float(__float_as_uint(x1) & 0xFFFF0000u);
+        const float r0 = x0 - h0, r1 = x1 - h1;
+        const float m0 = __uint_as_float(__float_as_uint(r0) & 0xFFFF0000u);
+        const float m1 = __uint_as_float(__float_as_uint(r1) & 0xFFFF0000u);
+        out[0] = (__float_as_uint(h0) >> 16) | (__float_as_uint(h1) & 0xFFFF0000u);
+        out[1] = (__float_as_uint(m0) >> 16) | (__float_as_uint(m1) & 0xFFFF0000u);
+        __nv_bfloat162 l = __floats2bfloat162_rn(r0 - m0, r1 - m1);
+        out[2] = *reinterpret_cast<uint32_t*>(&l);
+    } else {
+        const float h0 = __uint_as_float(__float_as_uint(x0) & 0xFFFFE000u);
+        const float h1 = __uint_as_float(__float_as_uint(x1) & 0xFFFFE000u);
+        __half2 h = __floats2half2_rn(h0, h1);
+        __half2 l = __floats2half2_rn(x0 - h0, x1 - h1);
+        out[0] = *reinterpret_cast<uint32_t*>(&h);
+        out[1] = *reinterpret_cast<uint32_t*>(&l);
+        out[2] = 0;
+    }
+}
+
+// ---------------------------------------------------------------- mbarrier + bulk copy
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// order this thread's generic-proxy shared-memory writes before later async-proxy (TMA) writes
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Bounded wait for the phase with parity `parity` to complete. Returns false after
+// `max_iter` unsuccessful polls (the caller records an error and stops waiting).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter = (1u << 26)) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t i = 0; i < max_iter; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// 1-D bulk copy global -> shared (TMA engine), completion counted on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------- fp16 magic
+// 0x6400 is fp16 1024.0: OR-ing a code u < 1024 into the mantissa gives 1024 + u.
+constexpr uint32_t MAGIC = 0x64006400u;
+
+template <int F>
+__device__ __forceinline__ uint32_t debias(uint32_t x) {
+    // (1024 + u) - (1024 + off) = u - off, exact
+    constexpr uint32_t bias_h = 0x6400u + (uint32_t)Fmt<F>::off;   // fp16 bits of 1024 + off (exact, off < 1024)
+    const __half2 b = __halves2half2(__ushort_as_half((unsigned short)bias_h), __ushort_as_half((unsigned short)bias_h));
+    __half2 v = *reinterpret_cast<__half2*>(&x);
+    __half2 r = __hsub2(v, b);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+}  // namespace mma
+}  // namespace kvq
+
+namespace kvq {
+namespace mma {
+
+// ---------------------------------------------------------------- K side (QK^T)
+// A operand of S^T = K Q^T for one 32-channel block b: rows are the sub-tile tokens
+// (g, g + 8), the k dimension runs over channels. Thread t (lane & 3) holds channels
+// 8t..8t+7 of the block; per MMA m in {0, 1} the k order is
+//   quantized: (8t+2m, 8t+2m+4, 8t+2m+1, 8t+2m+5)   16-bit float: 8t+4m+{0,1,2,3}
+// (q_channel gives the same order to the query operand).
+template <int F>
+__device__ __forceinline__ int q_channel(int t, int m, int slot) {
+    if constexpr (Fmt<F>::is_float) return 8 * t + 4 * m + slot;
+    else return 8 * t + 2 * m + ((slot & 1) ? 4 : 0) + (slot >> 1);
+}
+
+// four code pairs (n_j, n_{j+4}) of 8 consecutive channels of one row, biased by 1024
+template <int F>
+__device__ __forceinline__ void k_pairs(const uint8_t* row, int nb, int b, int t, uint32_t (&p)[4]) {
+    using FT = Fmt<F>;
+    constexpr int w0 = FT::w0, w1 = FT::w1;
+    const uint8_t* p0 = row + FT::off_p0(nb);
+    if constexpr (w0 == 4) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p0 + 16 * b + 4 * t);
+        p[0] = and_or(w, 0x000F000Fu, MAGIC);
+        p[1] = and_or(w >> 4, 0x000F000Fu, MAGIC);
+        p[2] = and_or(w >> 8, 0x000F000Fu, MAGIC);
+        p[3] = and_or(w >> 12, 0x000F000Fu, MAGIC);
+    } else if constexpr (w0 == 8) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p0 + 32 * b + 8 * t);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[j] = and_or(prmt(w.x, w.y, (uint32_t)(j | ((4 + j) << 8))), 0x00FF00FFu, MAGIC);
+    } else {  // w0 == 2
+        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p0 + 8 * b + 2 * t);
+        const uint32_t x = prmt(hw, 0u, 0x4140u);
+        p[0] = and_or(x, 0x00030003u, MAGIC);
+        p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
+        p[2] = and_or(x >> 4, 0x00030003u, MAGIC);
+        p[3] = and_or(x >> 6, 0x00030003u, MAGIC);
+    }
+    if constexpr (w1 == 2) {
+        const uint8_t* p1 = row + FT::off_p1(nb);
+        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p1 + 8 * b + 2 * t);
+        const uint32_t x = prmt(hw, 0u, 0x4140u);
+        constexpr uint32_t M = 0x00030003u << w0;
+        p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
+        p[1] = and_or(shift<w0 - 2>(x), M, p[1]);
+        p[2] = and_or(shift<w0 - 4>(x), M, p[2]);
+        p[3] = and_or(shift<w0 - 6>(x), M, p[3]);
+    } else if constexpr (w1 == 1) {
+        const uint8_t* p1 = row + FT::off_p1(nb);
+        const uint32_t by = p1[4 * b + t];
+        const uint32_t x = by | (by << 12);
+        constexpr uint32_t M = 0x00010001u << w0;
+        p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
+        p[1] = and_or(shift<w0 - 1>(x), M, p[1]);
+        p[2] = and_or(shift<w0 - 2>(x), M, p[2]);
+        p[3] = and_or(shift<w0 - 3>(x), M, p[3]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) p[j] = debias<F>(p[j]);
+}
+
+template <int F>
+__device__ __forceinline__ void k_frags(const uint8_t* rg, const uint8_t* rg8, int nb, int b, int t,
+                                        uint32_t (&a)[2][4]) {
+    if constexpr (Fmt<F>::is_float) {
+        const uint4 x = *reinterpret_cast<const uint4*>(rg + 64 * b + 16 * t);
+        const uint4 y = *reinterpret_cast<const uint4*>(rg8 + 64 * b + 16 * t);
+        a[0][0] = x.x; a[0][1] = y.x; a[0][2] = x.y; a[0][3] = y.y;
+        a[1][0] = x.z; a[1][1] = y.z; a[1][2] = x.w; a[1][3] = y.w;
+    } else {
+        uint32_t pg[4], pg8[4];
+        k_pairs<F>(rg, nb, b, t, pg);
+        k_pairs<F>(rg8, nb, b, t, pg8);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            a[m][0] = pg[2 * m];
+            a[m][1] = pg8[2 * m];
+            a[m][2] = pg[2 * m + 1];
+            a[m][3] = pg8[2 * m + 1];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- V side (P V)
+// A operand of O^T = V^T P^T for block b: rows are channels, the k dimension runs over
+// the sub-tile tokens (2t, 2t+1, 2t+8, 2t+9) held by thread (g, t). Thread g covers
+// channels 8k + 4hs + i (k = g >> 1, hs = g & 1, i = 0..3); in M-tile mt row g is
+// channel 8k + 4hs + 2mt and row g + 8 is channel 8k + 4hs + 2mt + 1.
+__device__ __forceinline__ int v_channel(int g, int mt, int row_hi) {
+    return 8 * (g >> 1) + 4 * (g & 1) + 2 * mt + row_hi;
+}
+
+// four channel pairs over two tokens (ra, rb): pair i = (token a, token b) of channel
+// 8k + 4hs + i, biased by 1024 (quantized) or raw 16-bit values (float formats)
+template <int F>
+__device__ __forceinline__ void v_pairs(const uint8_t* ra, const uint8_t* rb, int nb, int b, int g,
+                                        uint32_t (&p)[4]) {
+    using FT = Fmt<F>;
+    constexpr int w0 = FT::w0, w1 = FT::w1;
+    const int k = g >> 1, hs = g & 1;
+    if constexpr (FT::is_float) {
+        const uint2 wa = *reinterpret_cast<const uint2*>(ra + 64 * b + 16 * k + 8 * hs);
+        const uint2 wb = *reinterpret_cast<const uint2*>(rb + 64 * b + 16 * k + 8 * hs);
+        p[0] = prmt(wa.x, wb.x, 0x5410u);
+        p[1] = prmt(wa.x, wb.x, 0x7632u);
+        p[2] = prmt(wa.y, wb.y, 0x5410u);
+        p[3] = prmt(wa.y, wb.y, 0x7632u);
+        return;
+    } else {
+        const int o0 = FT::off_p0(nb);
+        if constexpr (w0 == 4) {
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + 16 * b + 4 * k);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + 16 * b + 4 * k);
+            const uint32_t x = prmt(wa, wb, hs ? 0x7632u : 0x5410u);
+            p[0] = and_or(x, 0x000F000Fu, MAGIC);
+            p[1] = and_or(x >> 4, 0x000F000Fu, MAGIC);
+            p[2] = and_or(x >> 8, 0x000F000Fu, MAGIC);
+            p[3] = and_or(x >> 12, 0x000F000Fu, MAGIC);
+        } else if constexpr (w0 == 8) {
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + 32 * b + 8 * k + 4 * hs);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + 32 * b + 8 * k + 4 * hs);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) p[i] = and_or(prmt(wa, wb, (uint32_t)(i | ((4 + i) << 8))), 0x00FF00FFu, MAGIC);
+        } else {  // w0 == 2
+            const uint32_t ba = ra[o0 + 8 * b + 2 * k + hs];
+            const uint32_t bb = rb[o0 + 8 * b + 2 * k + hs];
+            const uint32_t x = prmt(ba, bb, 0x5410u);
+            p[0] = and_or(x, 0x00030003u, MAGIC);
+            p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
+            p[2] = and_or(x >> 4, 0x00030003u, MAGIC);
+            p[3] = and_or(x >> 6, 0x00030003u, MAGIC);
+        }
+        if constexpr (w1 == 2) {
+            const int o1 = FT::off_p1(nb);
+            const uint32_t ha = ra[o1 + 8 * b + 2 * k + hs];
+            const uint32_t hb = rb[o1 + 8 * b + 2 * k + hs];
+            const uint32_t y = prmt(ha, hb, 0x5410u);
+            constexpr uint32_t M = 0x00030003u << w0;
+            p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
+            p[1] = and_or(shift<w0 - 2>(y), M, p[1]);
+            p[2] = and_or(shift<w0 - 4>(y), M, p[2]);
+            p[3] = and_or(shift<w0 - 6>(y), M, p[3]);
+        } else if constexpr (w1 == 1) {
+            const int o1 = FT::off_p1(nb);
+            const uint32_t ha = ra[o1 + 4 * b + k];
+            const uint32_t hb = rb[o1 + 4 * b + k];
+            const uint32_t y = prmt(ha, hb, 0x5410u) >> (4 * hs);
+            constexpr uint32_t M = 0x00010001u << w0;
+            p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
+            p[1] = and_or(shift<w0 - 1>(y), M, p[1]);
+            p[2] = and_or(shift<w0 - 2>(y), M, p[2]);
+            p[3] = and_or(shift<w0 - 3>(y), M, p[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = debias<F>(p[i]);
+    }
+}
+
+// tokens r0..r3 = sub-tile rows 2t, 2t+1, 2t+8, 2t+9 (rows past the data hold finite
+// stale values; their P entries are zero)
+template <int F>
+__device__ __forceinline__ void v_frags(const uint8_t* r0, const uint8_t* r1, const uint8_t* r2, const uint8_t* r3,
+                                        int nb, int b, int g, uint32_t (&a)[2][4]) {
+    uint32_t pa[4], pb[4];
+    v_pairs<F>(r0, r1, nb, b, g, pa);
+    v_pairs<F>(r2, r3, nb, b, g, pb);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        a[mt][0] = pa[2 * mt];
+        a[mt][1] = pa[2 * mt + 1];
+        a[mt][2] = pb[2 * mt];
+        a[mt][3] = pb[2 * mt + 1];
+    }
+}
+
+// Quantized V with the block scale folded into the A operand: for the token pairs
+// (r0, r1) and (r2, r3), x = d * (u - off) is computed in fp16 as hi = RN(d * c) and the
+// exact remainder lo = d * c - hi (fused multiply-add, single rounding; d * c has at most
+// 17 significant bits, so hi + lo == d * c unless the fp16 subnormal range is reached).
+template <int F>
+__device__ __forceinline__ void v_frags_scaled(const uint8_t* r0, const uint8_t* r1, const uint8_t* r2,
+                                               const uint8_t* r3, int nb, int b, int g,
+                                               uint32_t (&ahi)[2][4], uint32_t (&alo)[2][4]) {
+    uint32_t pa[4], pb[4];
+    v_pairs<F>(r0, r1, nb, b, g, pa);
+    v_pairs<F>(r2, r3, nb, b, g, pb);
+    const uint32_t d01 = prmt(reinterpret_cast<const uint16_t*>(r0)[b], reinterpret_cast<const uint16_t*>(r1)[b], 0x5410u);
+    const uint32_t d23 = prmt(reinterpret_cast<const uint16_t*>(r2)[b], reinterpret_cast<const uint16_t*>(r3)[b], 0x5410u);
+    const __half2 da = *reinterpret_cast<const __half2*>(&d01);
+    const __half2 db = *reinterpret_cast<const __half2*>(&d23);
+    uint32_t ha[4], la[4], hb[4], lb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 xa = *reinterpret_cast<const __half2*>(&pa[i]);
+        const __half2 xb = *reinterpret_cast<const __half2*>(&pb[i]);
+        const __half2 h1 = __hmul2_rn(xa, da);
+        const __half2 h2 = __hmul2_rn(xb, db);
+        const __half2 l1 = __hfma2(xa, da, __hneg2(h1));
+        const __half2 l2 = __hfma2(xb, db, __hneg2(h2));
+        ha[i] = *reinterpret_cast<const uint32_t*>(&h1);
+        hb[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        la[i] = *reinterpret_cast<const uint32_t*>(&l1);
+        lb[i] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        ahi[mt][0] = ha[2 * mt]; ahi[mt][1] = ha[2 * mt + 1]; ahi[mt][2] = hb[2 * mt]; ahi[mt][3] = hb[2 * mt + 1];
+        alo[mt][0] = la[2 * mt]; alo[mt][1] = la[2 * mt + 1]; alo[mt][2] = lb[2 * mt]; alo[mt][3] = lb[2 * mt + 1];
+    }
+}
+
+}  // namespace mma
+}  // namespace kvq
