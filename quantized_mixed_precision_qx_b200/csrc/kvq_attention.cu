@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, 
     const long long stride = (long long)G * (D + 2);
     const float* base = ws + ((br * H + h) * n_split) * stride;
     const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the preceding pass(es)
 
     float M = -INFINITY;
     for (int s = tid; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * stride + g]);
@@ -289,6 +290,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     const long long n_main = n - n_ring;
     const int CPL = lv.D / 32;
     const bool tcp = use_tensor_cores(lv.D);
+    int launched = 0;
     for (int region = 0; region < 2; ++region) {
         a.ring = region;
         a.chunk = region ? plan.ring_chunk : plan.main_chunk;
@@ -323,6 +325,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
             t.H = lv.H;
             t.G = lv.G;
             t.D = lv.D;
+            t.dependent = launched ? 1 : 0;
             const dim3 grid(ns, lv.H, lv.B * rows);
             e = tc::launch_tc(fk.id, fv.id, t, grid, tc::smem_bytes(fk.stride, fv.stride, lv.D), st);
         } else {
@@ -335,9 +338,21 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
             }
         }
         if (e != cudaSuccess) return e;
+        ++launched;
     }
-    const dim3 grid((unsigned)((long long)lv.B * rows * lv.H * lv.G), (unsigned)((lv.D + 31) / 32));
-    attn_merge<<<grid, 256, (size_t)a.n_split * sizeof(float), st>>>(ws, out, lv.G, lv.H, lv.D, a.n_split);
+    // the merge is a programmatic dependent: it launches early and waits for the passes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((long long)lv.B * rows * lv.H * lv.G), (unsigned)((lv.D + 31) / 32));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = (size_t)a.n_split * sizeof(float);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_merge, (const float*)ws, out, lv.G, lv.H, lv.D, a.n_split);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -46,6 +46,11 @@ struct Args {
     long long region_stride_k, region_stride_v;   // bytes between (b, h) regions
     int split_offset, n_split;
     int H, G, D;
+    // 0: first launch of the call (lets the next launch start early);
+    // 1: launched as a programmatic dependent of the previous pass: runs concurrently
+    //    with it and, before exiting, waits for it to finish, so a later dependent that
+    //    waits on this grid also sees the earlier one's results
+    int dependent;
 };
 
 __host__ __device__ constexpr size_t stage_bytes(int ks, int vs) { return (size_t)TOK * (ks + vs); }
@@ -105,6 +110,7 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     const float* sK = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 0) * D : nullptr;
     const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
 
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], CWARPS); }
         *fault = 0;
@@ -420,6 +426,7 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
         part[2 * G + idx] = O;
         if (c == 0) { part[hh] = M; part[G + hh] = L; }
     }
+    if (a.dependent) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace tc

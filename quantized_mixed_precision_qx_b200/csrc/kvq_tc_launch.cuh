@@ -8,14 +8,25 @@ namespace tc {
 
 template <int KF, int VF, int NB>
 cudaError_t launch_nb(const Args& a, dim3 grid, size_t smem, cudaStream_t st) {
-    static bool attr = false;      // raise the dynamic shared memory limit once per kernel
-    if (!attr) {
+    static bool smem_raised = false;      // raise the dynamic shared memory limit once per kernel
+    if (!smem_raised) {
         cudaError_t e = cudaFuncSetAttribute(decode_tc<KF, VF, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              227 * 1024);
         if (e != cudaSuccess) return e;
-        attr = true;
+        smem_raised = true;
     }
-    decode_tc<KF, VF, NB><<<grid, THREADS, smem, st>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.dependent ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc<KF, VF, NB>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
