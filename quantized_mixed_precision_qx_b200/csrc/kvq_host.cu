@@ -245,6 +245,20 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const float* q, flo
 kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, int32_t n_chunk, float scale,
                                  float* out, void* ws, size_t ws_bytes, void* stream) {
     if (n_chunk < 1) return KVQ_ERR_INVALID_ARG;
+    if (c && prefill_supported(c->L.head_dim)) {
+        // tensor-core path: validated like the split-K path, needs no workspace
+        if (layer < 0 || layer >= c->L.n_layers || !q || !out || !ws) return KVQ_ERR_INVALID_ARG;
+        if (!c->buf) return KVQ_ERR_NOT_BOUND;
+        if (!aligned16(q) || !aligned16(out) || !aligned16(ws)) return KVQ_ERR_ALIGNMENT;
+        const long long n = c->n[layer];
+        if (n == 0) return KVQ_ERR_EMPTY;
+        if (n_chunk > n) return KVQ_ERR_INVALID_ARG;
+        size_t need = 0;
+        kvq_status s = kvq_decode_workspace_bytes(c, n_chunk, &need);
+        if (s != KVQ_OK) return s;
+        if (ws_bytes < need) return KVQ_ERR_CAPACITY;
+        return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream));
+    }
     return attention_common(c, layer, q, n_chunk, scale, out, ws, ws_bytes, stream);
 }
 

@@ -113,4 +113,10 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
                              float* ws, long long n, int rows, const SplitPlan& plan,
                              cudaStream_t st);
 
+// Chunked prefill on tcgen05 (head_dim 128 / 256): q, out [B][C][Hq][D], n = cached
+// positions after the chunk's append.
+bool prefill_supported(int D);
+cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
+                           cudaStream_t st);
+
 }  // namespace kvq

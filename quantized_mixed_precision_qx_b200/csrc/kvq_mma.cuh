@@ -142,18 +142,29 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
     asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}"
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
-// Bounded wait for the phase with parity `parity` to complete. Returns false after
-// `max_iter` unsuccessful polls (the caller records an error and stops waiting).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter = (1u << 26)) {
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for the phase with parity `parity` to complete. Returns false once about
+// `limit_ns` nanoseconds have passed without completion (the caller records an error and
+// stops waiting), so a wait that can never finish ends the kernel instead of hanging it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
     const uint32_t a = smem_u32(bar);
-    for (uint32_t i = 0; i < max_iter; ++i) {
+    uint64_t start = 0;
+    for (uint32_t i = 0;; ++i) {
         uint32_t done;
         asm volatile(
             "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
             : "=r"(done) : "r"(a), "r"(parity) : "memory");
         if (done) return true;
+        if ((i & 63) == 0) {
+            const uint64_t now = global_ns();
+            if (i == 0) start = now;
+            else if (now - start > limit_ns) return false;
+        }
     }
-    return false;
 }
 // 1-D bulk copy global -> shared (TMA engine), completion counted on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.

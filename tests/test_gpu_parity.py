@@ -157,3 +157,23 @@ def test_error_paths_gpu():
     with pytest.raises(kvq.KVQError) as e:
         kvq.kvq_decode_attention(g.handle, 0, q, 1.0, out, g.ws, 4)
     assert e.value.status == kvq.ERR_CAPACITY
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("tail,W", [(orc.NONE, 0), (orc.Q8_0, 96), (orc.BF16, 40), (orc.F16, 300)])
+def test_prefill_formats(D, tail, W):
+    """Tensor-core prefill: chunks longer and shorter than the window, ragged row
+    counts (C * G not a multiple of 128), symmetric and asymmetric formats, KVarN."""
+    for kf, vf, kvarn, G in [(orc.Q6_0, orc.Q5_0, 0, 6), (orc.Q4_1, orc.Q3_1, 0, 8), (orc.Q8_0, orc.Q2_1, 1, 3),
+                             (orc.Q5_1, orc.Q8_1, 0, 1)]:
+        H = 2
+        T = 700
+        wl = Workload(1, 1, H, H * G, D, T, KVRecipe("outlier" if kf % 2 == 0 else "offset"), seed=40 + kf)
+        g, o = make_pair(wl, kf, vf, tail, W, kvarn=kvarn, calib=64)
+        vmax = append_both(g, o, wl, 0, 0, 517)
+        vmax = max(vmax, append_both(g, o, wl, 0, 517, T))
+        C = T - 517
+        q = wl.q_prefill(0, C)
+        out = g.prefill(0, to_dev(q), 0.75).cpu().numpy()
+        ref = o.prefill(0, q, 0.75)
+        check_close(out, ref, vmax, f"prefill kf={kf} vf={vf} tail={tail} W={W} D={D} kvarn={kvarn}")
