@@ -133,7 +133,7 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     const int b = (int)(bi / C);
     const int D = lv.D;
     const float* src = (kv ? v : k) + (((long long)b * C + i) * lv.H + h) * D;
-    const RowFmt& fl = lv.fmt[kv];
+    const RowFmt fl = kv ? lv.fmt[1] : lv.fmt[0];   // by value: no pointer into the parameters
     uint8_t* main = lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv];
     const float* s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * D : nullptr;
     const long long p = n + i;

@@ -6,7 +6,9 @@
 // with fp32 accumulators in tensor memory:
 //
 //   CTA   = 128 query rows of one (batch, kv head): row r = chunk row * G + head in group,
-//           TMEM lane r; 4 warps, one thread per row.
+//           TMEM lane r. 8 warps: warps 0-3 own one row per thread (softmax, epilogue);
+//           all 8 share the dequantization; its global loads run under the MMAs, with every load
+//           of a phase issued before its values are used.
 //   tile  = 64 key positions. Each tile is dequantized into shared memory as exact fp16
 //           hi + lo parts (K~ = hi + lo; the query and P are split the same way), and
 //           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N64 K16 steps) -> TMEM cols [0, 64)
@@ -25,7 +27,7 @@ namespace {
 
 constexpr int PM = 128;           // query rows per CTA
 constexpr int PN = 64;            // key positions per tile
-constexpr int PTHREADS = 128;
+constexpr int PTHREADS = 256;     // 8 warps: warps 0-3 own the 128 TMEM rows, all dequantize
 constexpr float PF_RESCALE = 8.0f;
 
 struct PrefillArgs {
@@ -39,44 +41,8 @@ struct PrefillArgs {
 };
 
 __host__ __device__ constexpr size_t pf_smem(int D) {
-    return 1024 /* alignment slack */ + 2 * (size_t)PM * D * 2 + 2 * (size_t)PN * D * 2 + 2 * (size_t)PM * PN * 2 + 64;
-}
-
-// value of channel c0 + j (j < 8) of a stored row; c0 % 8 == 0
-__device__ __forceinline__ void decode8(const uint8_t* __restrict__ row, const RowFmt& f, int c0, float (&x)[8]) {
-    if (f.kind != 0) {
-        const uint4 w = *reinterpret_cast<const uint4*>(row + 2 * c0);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (f.kind == 1) {
-                x[2 * j] = __uint_as_float(ws[j] << 16);
-                x[2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
-            } else {
-                x[2 * j] = mma::h2f_lo(ws[j]);
-                x[2 * j + 1] = mma::h2f_hi(ws[j]);
-            }
-        }
-        return;
-    }
-    const int blk = c0 >> 5;
-    const float d = mma::h2f_lo(reinterpret_cast<const uint16_t*>(row)[blk]);
-    const float m = f.asym ? mma::h2f_lo(reinterpret_cast<const uint16_t*>(row + f.off_m)[blk]) : 0.f;
-    uint64_t p0;
-    const uint8_t* a0 = row + f.off_p0 + c0 * f.w0 / 8;
-    if (f.w0 == 8) p0 = *reinterpret_cast<const unsigned long long*>(a0);
-    else if (f.w0 == 4) p0 = *reinterpret_cast<const uint32_t*>(a0);
-    else p0 = *reinterpret_cast<const uint16_t*>(a0);
-    uint32_t p1 = 0;
-    if (f.w1 == 2) p1 = *reinterpret_cast<const uint16_t*>(row + f.off_p1 + c0 / 4);
-    else if (f.w1 == 1) p1 = row[f.off_p1 + c0 / 8];
-    const uint32_t m0 = (1u << f.w0) - 1, m1 = (1u << f.w1) - 1;
-    const int off = 1 << (f.bits - 1);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int u = (int)(((uint32_t)(p0 >> (j * f.w0)) & m0) | (((p1 >> (j * f.w1)) & m1) << f.w0));
-        x[j] = f.asym ? __fadd_rn(__fmul_rn(d, (float)u), m) : __fmul_rn(d, (float)(u - off));
-    }
+    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 65536 /* staging */ +
+           2 * (size_t)PN * D * 2 + 2 * (size_t)PM * PN * 2 + 64;
 }
 
 // split fp32 -> fp16 hi (truncated to 11 significant bits) + fp16 lo (rounded remainder)
@@ -97,195 +63,501 @@ __device__ __forceinline__ void store_chunk(uint8_t* hi_tile, uint8_t* lo_tile, 
     *reinterpret_cast<uint4*>(lo_tile + off) = *reinterpret_cast<const uint4*>(l);
 }
 
-// stored row of position t (low-bit store or ring) and whether KVarN scales apply
-__device__ __forceinline__ const uint8_t* position_row(const LayerView& lv, int b, int h, int kv, long long t,
-                                                       long long n, const RowFmt*& f, const float*& s) {
-    const long long W = lv.W;
-    if (W > 0 && t >= n - W) {
-        f = &lv.tail;
-        s = nullptr;
-        return lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region + (t % W) * lv.tail.stride;
-    }
-    f = &lv.fmt[kv];
-    s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * lv.D : nullptr;
-    return lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv] + t * lv.fmt[kv].stride;
+// Per-kernel copy (registers) of what the dequantization needs; built from the launch
+// parameters once, so no field is ever read through a pointer into the parameter block.
+struct SideView {
+    const uint8_t* main;          // region of this (b, h)
+    const uint8_t* ring;
+    const float* scales;          // KVarN scales of this (b, h), or null
+    RowFmt fmain, ftail;
+    int W;
+};
+
+__device__ __forceinline__ SideView side_view(const LayerView& lv, int b, int h, int kv) {
+    SideView v;
+    v.main = lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv];
+    v.ring = lv.W ? lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region : nullptr;
+    v.scales = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * lv.D : nullptr;
+    v.fmain = lv.fmt[kv];
+    v.ftail = lv.tail;
+    v.W = lv.W;
+    return v;
 }
+
+// Raw words of channels c0..c0+7 of one stored row, fetched with loads that do not depend
+// on each other (so a thread can have many rows in flight) and decoded afterwards.
+struct Raw8 {
+    uint64_t w;        // 8-byte-aligned window holding plane 0 (low-bit) / channels c0..c0+3 (16-bit)
+    uint64_t w2;       // channels c0+4..c0+7 (16-bit rows only)
+    uint32_t p1;       // 2-byte window holding plane 1
+    uint32_t dm;       // d (low 16 bits), m (high 16 bits)
+    uint32_t sh0, sh1; // bit offsets of the fields inside w / p1
+    uint32_t sel;      // 0 = low-bit main row, 1 = tail row
+};
+
+// same, for a row already located (e.g. in the staging buffer) with its format
+__device__ __forceinline__ void fetch8_row(const uint8_t* row, const RowFmt f, uint32_t sel, int c0, Raw8& r) {
+    r.sel = sel;
+    if (f.kind != 0) {
+        const uint8_t* a = row + 2 * c0;                       // 16-byte aligned
+        r.w = *reinterpret_cast<const unsigned long long*>(a);
+        r.w2 = *reinterpret_cast<const unsigned long long*>(a + 8);
+        r.p1 = 0; r.dm = 0; r.sh0 = 0; r.sh1 = 0;
+        return;
+    }
+    const int blk = c0 >> 5;
+    const uint32_t d = reinterpret_cast<const uint16_t*>(row)[blk];
+    const uint32_t m = f.asym ? reinterpret_cast<const uint16_t*>(row + f.off_m)[blk] : 0u;
+    r.dm = d | (m << 16);
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(row + f.off_p0 + c0 * f.w0 / 8);
+    r.w = *reinterpret_cast<const unsigned long long*>(a0 & ~(uintptr_t)7);
+    r.sh0 = (uint32_t)(a0 & 7) * 8;
+    r.w2 = 0;
+    if (f.w1) {
+        const uintptr_t a1 = reinterpret_cast<uintptr_t>(row + f.off_p1 + c0 * f.w1 / 8);
+        r.p1 = *reinterpret_cast<const uint16_t*>(a1 & ~(uintptr_t)1);
+        r.sh1 = (uint32_t)(a1 & 1) * 8;
+    } else {
+        r.p1 = 0; r.sh1 = 0;
+    }
+}
+
+// decode fetched words to the values attention reads (KVarN scale applied to low-bit rows)
+__device__ __forceinline__ void decode_raw8(const SideView& v, const Raw8& r, int c0, float (&x)[8]) {
+    const RowFmt f = r.sel ? v.ftail : v.fmain;
+    if (f.kind != 0) {
+        const uint32_t w0 = (uint32_t)r.w, w1 = (uint32_t)(r.w >> 32), w2 = (uint32_t)r.w2, w3 = (uint32_t)(r.w2 >> 32);
+        if (f.kind == 1) {
+            x[0] = __uint_as_float(w0 << 16); x[1] = __uint_as_float(w0 & 0xFFFF0000u);
+            x[2] = __uint_as_float(w1 << 16); x[3] = __uint_as_float(w1 & 0xFFFF0000u);
+            x[4] = __uint_as_float(w2 << 16); x[5] = __uint_as_float(w2 & 0xFFFF0000u);
+            x[6] = __uint_as_float(w3 << 16); x[7] = __uint_as_float(w3 & 0xFFFF0000u);
+        } else {
+            x[0] = mma::h2f_lo(w0); x[1] = mma::h2f_hi(w0); x[2] = mma::h2f_lo(w1); x[3] = mma::h2f_hi(w1);
+            x[4] = mma::h2f_lo(w2); x[5] = mma::h2f_hi(w2); x[6] = mma::h2f_lo(w3); x[7] = mma::h2f_hi(w3);
+        }
+        return;
+    }
+    const float d = mma::h2f_lo(r.dm);
+    const float m = mma::h2f_hi(r.dm);
+    const uint64_t p0 = r.w >> r.sh0;
+    const uint32_t p1 = r.p1 >> r.sh1;
+    const uint32_t m0 = (1u << f.w0) - 1, m1 = (1u << f.w1) - 1;
+    const int off = 1 << (f.bits - 1);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int u = (int)(((uint32_t)(p0 >> (j * f.w0)) & m0) | (((p1 >> (j * f.w1)) & m1) << f.w0));
+        x[j] = f.asym ? __fadd_rn(__fmul_rn(d, (float)u), m) : __fmul_rn(d, (float)(u - off));
+    }
+    if (v.scales && !r.sel) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(v.scales[c0 + j], x[j]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fast dequantization for symmetric formats (qX_0, q8_0 tail) and the f16 tail: codes
+// become exact fp16 integers with the 1024-magic unpack of the decode kernel, and the
+// block scale is applied in fp16 as hi = RN(d*c), lo = d*c - hi (exact: d*c has at most
+// 17 significant bits). K chunks come out in the k order (c0, c4, c1, c5, c2, c6, c3, c7)
+// of each 8-channel chunk (the query is stored in the same order).
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr bool fast_fmt(int f) {
+    return f == F_Q2_0 || f == F_Q3_0 || f == F_Q4_0 || f == F_Q5_0 || f == F_Q6_0 || f == F_Q8_0 || f == F_F16;
+}
+
+__device__ __forceinline__ void scale_pairs(const uint32_t (&p)[4], uint32_t dpair, uint32_t (&hi)[4],
+                                            uint32_t (&lo)[4]) {
+    const __half2 d2 = *reinterpret_cast<const __half2*>(&dpair);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __half2 x = *reinterpret_cast<const __half2*>(&p[j]);
+        const __half2 h = __hmul2_rn(x, d2);
+        const __half2 l = __hfma2(x, d2, __hneg2(h));
+        hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[j] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+}
+
+// K: channels 32b + 8t .. +7 of one row -> hi/lo in k order (0,4,1,5,2,6,3,7)
+template <int F, int NB>
+__device__ __forceinline__ void k_chunk_fast(const uint8_t* row, int b, int t, uint32_t (&out)[8]) {
+    using namespace mma;
+    if constexpr (F == F_F16) {
+        const uint4 w = *reinterpret_cast<const uint4*>(row + 64 * b + 16 * t);
+        out[0] = prmt(w.x, w.z, 0x5410u); out[1] = prmt(w.x, w.z, 0x7632u);
+        out[2] = prmt(w.y, w.w, 0x5410u); out[3] = prmt(w.y, w.w, 0x7632u);
+        out[4] = out[5] = out[6] = out[7] = 0u;
+    } else {
+        uint32_t p[4], hi[4], lo[4];
+        k_pairs<F>(row, NB, b, t, p);
+        const uint32_t d = reinterpret_cast<const uint16_t*>(row)[b];
+        scale_pairs(p, d | (d << 16), hi, lo);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { out[j] = hi[j]; out[4 + j] = lo[j]; }
+    }
+}
+
+// V: channels 32b + 4g .. +3 at 8 positions (rows r[0..7]) -> per channel 8 positions
+// of hi (out[i][0..3]) and lo (out[i][4..7])
+template <int F, int NB>
+__device__ __forceinline__ void v_chunk_fast(const uint8_t* const (&r)[8], int b, int g, uint32_t (&out)[4][8]) {
+    using namespace mma;
+#pragma unroll
+    for (int pp = 0; pp < 4; ++pp) {
+        uint32_t p[4];
+        v_pairs<F>(r[2 * pp], r[2 * pp + 1], NB, b, g, p);
+        if constexpr (F == F_F16) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { out[i][pp] = p[i]; out[i][4 + pp] = 0u; }
+        } else {
+            const uint32_t da = reinterpret_cast<const uint16_t*>(r[2 * pp])[b];
+            const uint32_t db = reinterpret_cast<const uint16_t*>(r[2 * pp + 1])[b];
+            uint32_t hi[4], lo[4];
+            scale_pairs(p, da | (db << 16), hi, lo);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { out[i][pp] = hi[i]; out[i][4 + pp] = lo[i]; }
+        }
+    }
+}
+
+// k order inside a K chunk: position p holds channel KPERM[p] of the chunk
+__device__ __forceinline__ void kperm8(const float (&x)[8], float (&y)[8]) {
+    y[0] = x[0]; y[1] = x[4]; y[2] = x[1]; y[3] = x[5]; y[4] = x[2]; y[5] = x[6]; y[6] = x[3]; y[7] = x[7];
+}
+
+// Staging of one tile's raw rows (K rows then V rows), filled by bulk copies: positions
+// below the window come from the low-bit store, the others from the ring (in position
+// order, the ring slot range split at its wrap).
+struct Stage {
+    int t0, t_last;               // positions held
+    int n_main;                   // rows from the low-bit store (positions t0 .. t0 + n_main - 1)
+};
+constexpr int STAGE_HALF = 32 * 1024;   // K rows at [0, 32 KB), V rows at [32 KB, 64 KB)
 
 template <int NB>
 __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     constexpr int D = 32 * NB;
+    constexpr int CHUNKS = D / 8;                    // 8-channel chunks per row
     const LayerView& lv = a.lv;
     extern __shared__ uint8_t raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* q_hi = sm;
-    uint8_t* q_lo = q_hi + PM * D * 2;
-    uint8_t* kv_hi = q_lo + PM * D * 2;              // K~ [PN x D], later V~^T [D x PN]
+    uint8_t* q_hi = sm;                              // Q hi [PM x D]; Q lo lives in TMEM
+    uint8_t* stage = q_hi + PM * D * 2;              // raw rows of the next tile (64 KB)
+    uint8_t* kv_hi = stage + 2 * STAGE_HALF;         // K~ [PN x D], later V~^T [D x PN]
     uint8_t* kv_lo = kv_hi + PN * D * 2;
     uint8_t* p_hi = kv_lo + PN * D * 2;              // P [PM x PN]
     uint8_t* p_lo = p_hi + PM * PN * 2;
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);   // MMA completion
+    uint64_t* sbar = mbar + 1;                                          // staging copies
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbar + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    const bool owner = tid < PM;                     // owns TMEM lane / query row tid
     const int G = lv.G, H = lv.H;
     const int h = blockIdx.y, b = blockIdx.z;
     const int rows_total = a.C * G;
-    const int r = blockIdx.x * PM + tid;             // query row of this thread
-    const bool row_ok = r < rows_total;
+    const int row0 = blockIdx.x * PM;
+    const int r = row0 + (tid & (PM - 1));           // query row of an owner thread
+    const bool row_ok = owner && r < rows_total;
     const int ci = row_ok ? r / G : 0;               // chunk row
     const int gi = row_ok ? r % G : 0;
-    const long long pos0 = a.n - a.C;
-    const long long my_limit = row_ok ? pos0 + ci : -1;   // last visible position
-    const int last_row = min(rows_total - 1, (int)blockIdx.x * PM + PM - 1);
-    const long long tile_limit = pos0 + last_row / G;      // last position any row sees
-    const long long first_row_limit = pos0 + ((int)blockIdx.x * PM) / G;
+    const int n = (int)a.n;                          // positions < 2^31 (checked on the host)
+    const int pos0 = n - a.C;
+    const int my_limit = row_ok ? pos0 + ci : -1;    // last visible position
+    const int last_row = min(rows_total - 1, row0 + PM - 1);
+    const int tile_limit = pos0 + last_row / G;      // last position any row sees
+    const int first_row_limit = pos0 + row0 / G;
+    const SideView kside = side_view(lv, b, h, 0);
+    const SideView vside = side_view(lv, b, h, 1);
+    const int W = lv.W;
+    const int ring0 = W > 0 ? n - W : n;             // first position held in the ring
+    const int n_tiles = tile_limit / PN + 1;
 
-    // ---- query rows -> Q hi/lo (scaled to base-2 logits)
-    {
-        const float* qr = a.q + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
-#pragma unroll 1
-        for (int k0 = 0; k0 < D; k0 += 8) {
-            float x[8];
-            if (row_ok) {
-                const float4 u = *reinterpret_cast<const float4*>(qr + k0);
-                const float4 v = *reinterpret_cast<const float4*>(qr + k0 + 4);
-                x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] *= a.qscale;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = 0.f;
-            }
-            store_chunk(q_hi, q_lo, tid, k0, PM, x);
-        }
+    if (tid == 0) {
+        mma::mbar_init(mbar, 1);
+        mma::mbar_init(sbar, 1);
+        mma::fence_mbar_init();
     }
-    if (tid == 0) { mma::mbar_init(mbar, 1); mma::fence_mbar_init(); }
     if (warp == 0) { t5::tmem_alloc(tmem_slot, 512); t5::tmem_relinquish(); }
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t t_s = tmem;                       // S: columns [0, 64)
-    const uint32_t t_o = tmem + 256;                 // O: columns [256, 512)
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t t_qlo = tmem + 64;                // Q lo: columns [64, 64 + D/2)
+    const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
 
-    const uint32_t idesc_s = t5::idesc_f16(PM, PN);
-    const uint32_t idesc_o = t5::idesc_f16(PM, D);
-    const uint32_t sq_hi = t5::smem_addr(q_hi), sq_lo = t5::smem_addr(q_lo);
-    const uint32_t skv_hi = t5::smem_addr(kv_hi), skv_lo = t5::smem_addr(kv_lo);
-    const uint32_t sp_hi = t5::smem_addr(p_hi), sp_lo = t5::smem_addr(p_lo);
+    // issue the bulk copies of tile `tile`'s raw rows into the staging buffer (thread 0)
+    auto issue_stage = [&](int tile) {
+        const int t0 = tile * PN;
+        const int tl = min(t0 + PN - 1, tile_limit);
+        const int nm = max(0, min(tl + 1, ring0) - t0);       // rows from the low-bit store
+        const int nr = (tl + 1 - t0) - nm;                    // rows from the ring
+        uint32_t bytes = 0;
+        for (int kv = 0; kv < 2; ++kv) {
+            const SideView& v = kv ? vside : kside;
+            uint8_t* dst = stage + kv * STAGE_HALF;
+            if (nm > 0) {
+                const uint32_t cb = (uint32_t)nm * v.fmain.stride;
+                bytes += cb;
+            }
+            if (nr > 0) bytes += (uint32_t)nr * v.ftail.stride;
+            (void)dst;
+        }
+        mma::mbar_arrive_expect_tx(sbar, bytes);
+        for (int kv = 0; kv < 2; ++kv) {
+            const SideView& v = kv ? vside : kside;
+            uint8_t* dst = stage + kv * STAGE_HALF;
+            if (nm > 0) {
+                const uint32_t cb = (uint32_t)nm * v.fmain.stride;
+                mma::bulk_g2s(dst, v.main + (long long)t0 * v.fmain.stride, cb, sbar);
+                dst += cb;
+            }
+            if (nr > 0) {
+                const int p = t0 + nm;                         // first ring position
+                const int s0 = p % W;
+                const int c1 = min(nr, W - s0);
+                mma::bulk_g2s(dst, v.ring + (long long)s0 * v.ftail.stride, (uint32_t)c1 * v.ftail.stride, sbar);
+                if (nr > c1)
+                    mma::bulk_g2s(dst + (size_t)c1 * v.ftail.stride, v.ring, (uint32_t)(nr - c1) * v.ftail.stride, sbar);
+            }
+        }
+    };
+    if (tid == 0) issue_stage(0);
 
-    float m_run = -INFINITY, l_run = 0.f;
-    uint32_t phase = 0;
-    bool have_o = false;
-    bool fault = false;
-    const long long n_tiles = tile_limit / PN + 1;
-
-    for (long long tile = 0; tile < n_tiles && !fault; ++tile) {
-        const long long t0 = tile * PN;
-        // ---------------- K~ tile -> hi/lo (rows = positions, k = channels); thread: half a row
-        {
-            const int tok = tid >> 1, half = tid & 1;
-            const long long t = t0 + tok;
-            const RowFmt* f;
-            const float* s;
-            const bool live = t <= tile_limit && t < a.n;
-            const uint8_t* row = live ? position_row(lv, b, h, 0, t, a.n, f, s) : nullptr;
+    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row)
+    if (owner) {
+        const float* qr = a.q + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
 #pragma unroll 1
-            for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 8) {
-                float x[8];
-                if (live) {
-                    decode8(row, *f, c0, x);
-                    if (s) {
+        for (int c64 = 0; c64 < D; c64 += 64) {      // 64 k-values = 32 TMEM columns
+            float cols[32];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(s[c0 + j], x[j]);
-                    }
+            for (int k0 = 0; k0 < 64; k0 += 8) {
+                float x[8], y[8];
+                if (row_ok) {
+                    const float4 p = *reinterpret_cast<const float4*>(qr + c64 + k0);
+                    const float4 v = *reinterpret_cast<const float4*>(qr + c64 + k0 + 4);
+                    x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w; x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) x[j] *= a.qscale;
                 } else {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) x[j] = 0.f;
                 }
-                store_chunk(kv_hi, kv_lo, tok, c0, PN, x);
+                kperm8(x, y);
+                __align__(16) __half hh[8], ll[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) split16(y[j], hh[j], ll[j]);
+                *reinterpret_cast<uint4*>(q_hi + t5::sw128_offset(tid, c64 + k0, PM)) = *reinterpret_cast<const uint4*>(hh);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    cols[k0 / 2 + j] = __uint_as_float((uint32_t)__half_as_ushort(ll[2 * j]) |
+                                                       ((uint32_t)__half_as_ushort(ll[2 * j + 1]) << 16));
+            }
+            t5::tmem_st32(t_qlo + lane_off + c64 / 2, cols);
+        }
+    }
+
+    const uint32_t idesc_s = t5::idesc_f16(PM, PN);
+    const uint32_t idesc_o = t5::idesc_f16(PM, D);
+    const uint32_t sq_hi = t5::smem_addr(q_hi);
+    const uint32_t skv_hi = t5::smem_addr(kv_hi), skv_lo = t5::smem_addr(kv_lo);
+    const uint32_t sp_hi = t5::smem_addr(p_hi), sp_lo = t5::smem_addr(p_lo);
+
+    // Tile modes (uniform over the CTA): 1 = every position in the low-bit store and its
+    // format has a fast path, 2 = every position in the ring with a fast tail format,
+    // 0 = generic decode (mixed tiles, asymmetric / bf16 formats, KVarN).
+    auto tile_mode = [&](int t0, const SideView& v) -> int {
+        const int last = min(t0 + PN - 1, tile_limit);
+        if (last < ring0 && !v.scales && fast_fmt(v.fmain.id)) return 1;
+        if (t0 >= ring0 && fast_fmt(v.ftail.id)) return 2;
+        return 0;
+    };
+    // staged row of position t (clamped to the tile's last position)
+    auto srow = [&](int kv, int t0, int t, uint32_t& sel) -> const uint8_t* {
+        const SideView& v = kv ? vside : kside;
+        const int tl = min(t0 + PN - 1, tile_limit);
+        t = min(t, tl);
+        const int nm = max(0, min(tl + 1, ring0) - t0);
+        const uint8_t* base = stage + kv * STAGE_HALF;
+        if (t - t0 < nm) { sel = 0; return base + (size_t)(t - t0) * v.fmain.stride; }
+        sel = 1;
+        return base + (size_t)nm * v.fmain.stride + (size_t)(t - t0 - nm) * v.ftail.stride;
+    };
+
+    float m_run = -INFINITY, l_run = 0.f;
+    uint32_t phase = 0, sphase = 0;
+    bool have_o = false;
+    bool fault = false;
+    constexpr int PER = PN * CHUNKS / PTHREADS;      // K chunk units per thread
+
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+
+    for (int tile = 0; tile < n_tiles && !fault; ++tile) {
+        const int t0 = tile * PN;
+        // ---------------- wait for the staged raw rows of this tile
+        fault = __syncthreads_or((!mma::mbar_wait(sbar, sphase & 1)) || fault) != 0;
+        ++sphase;
+        if (fault) break;
+        // ---------------- K~ tile -> hi/lo (rows = positions, k = channels in chunk k order)
+        {
+            const int kmode = tile_mode(t0, kside);
+            const int fid = kmode == 1 ? kside.fmain.id : kside.ftail.id;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int u = tid + i * PTHREADS;
+                const int kr = u / CHUNKS, ch = u % CHUNKS;
+                uint32_t sel;
+                const uint8_t* row = srow(0, t0, t0 + kr, sel);
+                uint32_t out[8];
+                if (kmode != 0) {
+                    const int cb = ch >> 2, ct = ch & 3;
+                    switch (fid) {
+                        case F_Q2_0: k_chunk_fast<F_Q2_0, NB>(row, cb, ct, out); break;
+                        case F_Q3_0: k_chunk_fast<F_Q3_0, NB>(row, cb, ct, out); break;
+                        case F_Q4_0: k_chunk_fast<F_Q4_0, NB>(row, cb, ct, out); break;
+                        case F_Q5_0: k_chunk_fast<F_Q5_0, NB>(row, cb, ct, out); break;
+                        case F_Q6_0: k_chunk_fast<F_Q6_0, NB>(row, cb, ct, out); break;
+                        case F_Q8_0: k_chunk_fast<F_Q8_0, NB>(row, cb, ct, out); break;
+                        default: k_chunk_fast<F_F16, NB>(row, cb, ct, out); break;
+                    }
+                    const uint32_t off = t5::sw128_offset(kr, 8 * ch, PN);
+                    *reinterpret_cast<uint4*>(kv_hi + off) = make_uint4(out[0], out[1], out[2], out[3]);
+                    *reinterpret_cast<uint4*>(kv_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
+                } else {
+                    Raw8 rk;
+                    fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, rk);
+                    float x[8], y[8];
+                    decode_raw8(kside, rk, 8 * ch, x);
+                    kperm8(x, y);
+                    store_chunk(kv_hi, kv_lo, kr, 8 * ch, PN, y);
+                }
             }
         }
         t5::fence_proxy_async();
         t5::fence_before_sync();
         __syncthreads();
         t5::fence_after_sync();
-        // ---------------- S = Q K~^T (3 passes)
+        // ---------------- S = Q K~^T: Qh Kh + Qh Kl (A from shared memory) + Ql Kh (A from TMEM)
         if (tid == 0) {
             int step = 0;
 #pragma unroll 1
-            for (int pass = 0; pass < 3; ++pass) {
-                const uint32_t qa = (pass == 2) ? sq_lo : sq_hi;
-                const uint32_t kb = (pass == 1) ? skv_lo : skv_hi;
+            for (int pass = 0; pass < 2; ++pass) {
+                const uint32_t kb = pass ? skv_lo : skv_hi;
 #pragma unroll 1
                 for (int k = 0; k < D / 16; ++k, ++step) {
-                    const uint64_t ad = t5::desc_sw128(qa + (k >> 2) * PM * 128 + (k & 3) * 32);
+                    const uint64_t ad = t5::desc_sw128(sq_hi + (k >> 2) * PM * 128 + (k & 3) * 32);
                     const uint64_t bd = t5::desc_sw128(kb + (k >> 2) * PN * 128 + (k & 3) * 32);
                     t5::mma_f16_ss(t_s, ad, bd, idesc_s, step > 0);
                 }
             }
+#pragma unroll 1
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t bd = t5::desc_sw128(skv_hi + (k >> 2) * PN * 128 + (k & 3) * 32);
+                t5::mma_f16_ts(t_s, t_qlo + 8 * k, bd, idesc_s, true);
+            }
             t5::mma_commit(mbar);
         }
+        // ---------------- V~ rows from the staging buffer into registers (during the MMAs)
+        const int vmode = tile_mode(t0, vside);
+        uint32_t xv[64];
+        if (vmode != 0) {
+            const int vfid = vmode == 1 ? vside.fmain.id : vside.ftail.id;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int u = tid + i * PTHREADS;    // (block, g, 8-position group)
+                if (u < NB * 64) {
+                    const int pg = u & 7, g = (u >> 3) & 7, vb = u >> 6;
+                    const uint8_t* rr[8];
+                    uint32_t sel;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) rr[j] = srow(1, t0, t0 + 8 * pg + j, sel);
+                    uint32_t o[4][8];
+                    switch (vfid) {
+                        case F_Q2_0: v_chunk_fast<F_Q2_0, NB>(rr, vb, g, o); break;
+                        case F_Q3_0: v_chunk_fast<F_Q3_0, NB>(rr, vb, g, o); break;
+                        case F_Q4_0: v_chunk_fast<F_Q4_0, NB>(rr, vb, g, o); break;
+                        case F_Q5_0: v_chunk_fast<F_Q5_0, NB>(rr, vb, g, o); break;
+                        case F_Q6_0: v_chunk_fast<F_Q6_0, NB>(rr, vb, g, o); break;
+                        case F_Q8_0: v_chunk_fast<F_Q8_0, NB>(rr, vb, g, o); break;
+                        default: v_chunk_fast<F_F16, NB>(rr, vb, g, o); break;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xv[32 * i + 8 * c + e] = o[c][e];
+                }
+            }
+        } else {
+            const int tg = tid % (PN / 8), cc = tid / (PN / 8);
+            if (cc < CHUNKS) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = t0 + 8 * tg + j;
+                    uint32_t sel;
+                    const uint8_t* row = srow(1, t0, t, sel);
+                    Raw8 rv;
+                    fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, rv);
+                    float x[8];
+                    decode_raw8(vside, rv, 8 * cc, x);
+                    const bool live = t <= tile_limit;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xv[8 * j + e] = __float_as_uint(live ? x[e] : 0.f);
+                }
+            }
+        }
+        // the staging buffer is free: fetch the next tile while this one finishes
+        mma::fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0 && tile + 1 < n_tiles) issue_stage(tile + 1);
         fault = __syncthreads_or((!mma::mbar_wait(mbar, phase & 1)) || fault) != 0;   // uniform
         ++phase;
         t5::fence_after_sync();
         // ---------------- V~ tile -> V~^T hi/lo (rows = channels, k = positions)
-        {
-            // thread: 8 positions x (D/16) channel chunks of 8 -> writes whole 16-byte chunks
-            const int tg = tid & 7;                  // position group: positions 8tg .. 8tg+7
-            const int cg = tid >> 3;                 // channel groups cg, cg+16, ...
-            const RowFmt* fr[8];
-            const float* sr[8];
-            const uint8_t* rowp[8];
-            bool live[8];
+        if (vmode != 0) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const long long t = t0 + 8 * tg + j;
-                live[j] = t <= tile_limit && t < a.n;
-                rowp[j] = live[j] ? position_row(lv, b, h, 1, t, a.n, fr[j], sr[j]) : nullptr;
-            }
-#pragma unroll 1
-            for (int cc = cg; cc < D / 8; cc += 16) {
-                float x[8][8];                       // [position][channel]
+            for (int i = 0; i < 2; ++i) {
+                const int u = tid + i * PTHREADS;
+                if (u < NB * 64) {
+                    const int pg = u & 7, g = (u >> 3) & 7, vb = u >> 6;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (live[j]) {
-                        decode8(rowp[j], *fr[j], 8 * cc, x[j]);
-                        if (sr[j]) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[j][e] = __fmul_rn(sr[j][8 * cc + e], x[j][e]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[j][e] = 0.f;
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t off = t5::sw128_offset(32 * vb + 4 * g + c, 8 * pg, D);
+                        const uint32_t* w = &xv[32 * i + 8 * c];
+                        *reinterpret_cast<uint4*>(kv_hi + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(kv_lo + off) = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 }
+            }
+        } else {
+            const int tg = tid % (PN / 8), cc = tid / (PN / 8);
+            if (cc < CHUNKS) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     float y[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) y[j] = x[j][e];
+                    for (int j = 0; j < 8; ++j) y[j] = __uint_as_float(xv[8 * j + e]);
                     store_chunk(kv_hi, kv_lo, 8 * cc + e, 8 * tg, D, y);
                 }
             }
         }
-        // ---------------- softmax on S (row-local)
-        {
-            float sv[PN];
-            float tmp[32];
-            t5::tmem_ld32(t_s + lane_off, tmp);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = tmp[i];
-            t5::tmem_ld32(t_s + lane_off + 32, tmp);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[32 + i] = tmp[i];
+        // ---------------- softmax on S (row owners; row-local)
+        if (owner) {
+            const bool full = t0 + PN - 1 <= first_row_limit;
             float mx = -INFINITY;
-            const bool full = t0 + PN - 1 <= first_row_limit && t0 + PN <= a.n;
 #pragma unroll
-            for (int i = 0; i < PN; ++i) {
-                if (!full && t0 + i > my_limit) sv[i] = -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+            for (int hc = 0; hc < PN; hc += 32) {
+                float sv[32];
+                t5::tmem_ld32(t_s + lane_off + hc, sv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float v = (!full && t0 + hc + i > my_limit) ? -INFINITY : sv[i];
+                    mx = fmaxf(mx, v);
+                }
             }
             const bool raise = mx > m_run + PF_RESCALE || (m_run == -INFINITY && mx > -INFINITY);
             const float corr = !raise ? 1.f : ((m_run == -INFINITY) ? 0.f : mma::ex2(m_run - mx));
@@ -307,19 +579,25 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             }
             float ps = 0.f;
 #pragma unroll
-            for (int i = 0; i < PN; ++i) {
-                const float p = (m_run == -INFINITY) ? 0.f : mma::ex2(sv[i] - m_run);
-                sv[i] = p;
-                ps += p;
+            for (int hc = 0; hc < PN; hc += 32) {
+                float sv[32];
+                t5::tmem_ld32(t_s + lane_off + hc, sv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool vis = full || t0 + hc + i <= my_limit;
+                    const float p = (m_run == -INFINITY || !vis) ? 0.f : mma::ex2(sv[i] - m_run);
+                    sv[i] = p;
+                    ps += p;
+                }
+#pragma unroll
+                for (int k0 = 0; k0 < 32; k0 += 8) {
+                    float x8[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) x8[j] = sv[k0 + j];
+                    store_chunk(p_hi, p_lo, tid, hc + k0, PM, x8);
+                }
             }
             l_run += ps;
-#pragma unroll
-            for (int k0 = 0; k0 < PN; k0 += 8) {
-                float x[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = sv[k0 + j];
-                store_chunk(p_hi, p_lo, tid, k0, PM, x);
-            }
         }
         t5::fence_proxy_async();
         t5::fence_before_sync();
@@ -347,9 +625,9 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         t5::fence_after_sync();
     }
 
-    // ---- epilogue: O / l -> out (TMEM loads by whole warps; only real rows store)
+    // ---- epilogue: O / l -> out (TMEM loads by whole owner warps; only real rows store)
     const bool any_fault = __syncthreads_or(fault ? 1 : 0) != 0;
-    if (have_o && !any_fault) {
+    if (owner && have_o && !any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         const float inv = row_ok ? 1.f / l_run : 0.f;
 #pragma unroll 1
@@ -366,6 +644,10 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     } else if (row_ok && any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
+    }
+    if (any_fault) {
+        // a copy may still be in flight into the staging buffer: give it a bounded wait
+        mma::mbar_wait(sbar, sphase & 1, 100000000ull);
     }
     t5::fence_before_sync();
     __syncthreads();
