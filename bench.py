@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -52,17 +53,20 @@ def decode_bytes(n: int) -> int:
     return rows + 2 * B_ * HQ_ * D_ * 4
 
 
-def append_bytes(n0: int, c: int) -> int:
+def append_bytes(n0: int, c: int, W: int = W_, rowk: int = ROW_K, rowv: int = ROW_V, rowt: int = ROW_T,
+                 B: int = B_, H: int = H_, D: int = D_) -> int:
     """Algorithmic bytes of appending c positions at context n0: fp32 K and V input,
     ring writes of the positions that end in the window, ring reads of evicted rows,
     and the low-bit rows written."""
+    if W == 0:
+        return B * H * c * (2 * D * 4 + rowk + rowv)
     n1 = n0 + c
-    in_ring = min(c, W_)                                  # new rows written to the ring
-    evicted = max(0, min(n0, n1 - W_) - max(0, n0 - W_))  # old ring rows requantized
-    direct = max(0, c - W_)                               # enter-and-leave rows
+    in_ring = min(c, W)                                   # new rows written to the ring
+    evicted = max(0, min(n0, n1 - W) - max(0, n0 - W))    # old ring rows requantized
+    direct = max(0, c - W)                                # enter-and-leave rows
     low = evicted + direct
-    per_bh = c * 2 * D_ * 4 + in_ring * 2 * ROW_T + evicted * 2 * ROW_T + low * (ROW_K + ROW_V)
-    return B_ * H_ * per_bh
+    per_bh = c * 2 * D * 4 + in_ring * 2 * rowt + evicted * 2 * rowt + low * (rowk + rowv)
+    return B * H * per_bh
 
 
 def read_peaks():
@@ -81,7 +85,9 @@ def source_hash(paths):
 
 
 DECODE_SOURCES = ["quantized_mixed_precision_qx_b200/csrc/kvq_attention.cu",
-                  "quantized_mixed_precision_qx_b200/csrc/kvq_rowio.cuh",
+                  "quantized_mixed_precision_qx_b200/csrc/kvq_decode_tc.cuh",
+                  "quantized_mixed_precision_qx_b200/csrc/kvq_mma.cuh",
+                  "quantized_mixed_precision_qx_b200/csrc/kvq_tc_launch.cuh",
                   "quantized_mixed_precision_qx_b200/csrc/kvq_internal.cuh"]
 
 
@@ -328,6 +334,7 @@ def run_kvq(args, rank, world):
     value = world * dec_bytes * args.steps / dec_t / 1e9
     achieved = dec_bytes * args.steps / dec_t / 1e9          # per GPU
     traffic = recorded_traffic()
+    extra = supplementary(dev, peak) if not args.no_extra else None
     cpu = None
     if world == 1:
         gbs, mtok, threads, desc, _ = oracle_sample(budget_s=15.0)
@@ -352,8 +359,130 @@ def run_kvq(args, rank, world):
                 "note": "decode bytes / whole step time with appends and host copies"},
         "gpu_launches": launches * args.steps,
         "clocks": clock_info,
+        "workloads": extra,
     }
     print(json.dumps(line), flush=True)
+
+
+def supplementary(dev, peak):
+    """Decode / append / prefill figures on the large workloads (one GPU, device-generated
+    seeded inputs; parity for these shapes is covered by the tests). Each decode is timed
+    with L2 flushed before it; caches are larger than L2 anyway."""
+    import torch
+    from quantized_mixed_precision_qx_b200 import kvq
+    res = {}
+    gen = torch.Generator(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def rows_bytes(fmt, D):
+        bb = {0: 10, 1: 12, 2: 14, 3: 16, 4: 18, 5: 20, 6: 22, 7: 24, 8: 26, 9: 28, 10: 34, 11: 36, 12: 64, 13: 64}[fmt]
+        return bb * D // 32
+
+    def fill(c, B, H, D, n, outlier=True, chunk=8192):
+        gen.manual_seed(1234)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        t = 0
+        scale = torch.ones(H, D, device=dev)
+        if outlier:
+            for h in range(H):
+                scale[h, torch.randperm(D, generator=gen, device=dev)[:8]] = 8.0
+        while t < n:
+            cc = min(chunk, n - t)
+            k = torch.randn(B, cc, H, D, device=dev, generator=gen) * scale
+            v = torch.randn(B, cc, H, D, device=dev, generator=gen)
+            torch.cuda.synchronize()
+            ev0.record()
+            c.append(0, k, v)
+            ev1.record()
+            torch.cuda.synchronize()
+            tot += ev0.elapsed_time(ev1) / 1e3
+            t += cc
+            del k, v
+        return tot
+
+    def time_decode(c, B, Hq, D, reps=10):
+        q = torch.randn(B, Hq, D, device=dev, generator=gen) / math.sqrt(D)
+        out = torch.empty_like(q)
+        ws = c.ensure_workspace(1)
+        ts = []
+        for i in range(reps + 3):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kvq.kvq_decode_attention(c.handle, 0, q, 1.0, out, ws, ws.numel())
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1) / 1e3)
+        return statistics.median(ts)
+
+    # full-length hybrid-model layer: fill 257,984, prefill 4,096, decode at 262,080
+    B, H, Hq, D, W = 1, 4, 24, 256, 2048
+    n_fill, C = 257984, 4096
+    c = kvq.KVCache(1, B, H, Hq, D, 262144, K_FMT, V_FMT, T_FMT, W, device=dev, ws_rows=C)
+    t_fill = fill(c, B, H, D, n_fill)
+    fill_bytes = sum(append_bytes(t, min(8192, n_fill - t), W, ROW_K, ROW_V, ROW_T, B, H, D)
+                     for t in range(0, n_fill, 8192))
+    gen.manual_seed(99)
+    kc = torch.randn(B, C, H, D, device=dev, generator=gen)
+    vc = torch.randn(B, C, H, D, device=dev, generator=gen)
+    c.append(0, kc, vc)
+    n = n_fill + C
+    q = torch.randn(B, C, Hq, D, device=dev, generator=gen) / math.sqrt(D)
+    out = torch.empty_like(q)
+    ws = c.ensure_workspace(C)
+    kvq.kvq_prefill_attention(c.handle, 0, q, C, 1.0, out, ws, ws.numel())
+    torch.cuda.synchronize()
+    pts = []
+    for _ in range(2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvq.kvq_prefill_attention(c.handle, 0, q, C, 1.0, out, ws, ws.numel())
+        e1.record()
+        torch.cuda.synchronize()
+        pts.append(e0.elapsed_time(e1) / 1e3)
+    keys = C * n_fill + C * (C + 1) / 2
+    pflop = keys * Hq * 4 * D
+    tp = min(pts)
+    td = time_decode(c, B, Hq, D)
+    dbytes = B * H * ((n - W) * (ROW_K + ROW_V) + W * 2 * ROW_T) + 2 * B * Hq * D * 4
+    res["full_length_layer"] = {
+        "decode_gbs": dbytes / td / 1e9, "decode_frac": dbytes / td / 1e9 / peak, "decode_us": td * 1e6,
+        "context": n, "append_fill_mtok_s": n_fill * B / t_fill / 1e6,
+        "append_fill_gbs": fill_bytes / t_fill / 1e9, "append_fill_frac": fill_bytes / t_fill / 1e9 / peak,
+        "prefill_ms": tp * 1e3, "prefill_alg_tflops": pflop / tp / 1e12,
+        "prefill_executed_tflops": 3 * pflop / tp / 1e12,
+        "note": "prefill FLOP = 4 x keys x heads x D (causal count); executed = 3 split-operand passes"}
+    del c, kc, vc, q, out, ws
+    torch.cuda.empty_cache()
+
+    # KVarN: batch 8, 2 kv heads, 131,072 positions
+    B, H, Hq, D, n = 8, 2, 16, 256, 131072
+    c = kvq.KVCache(1, B, H, Hq, D, n, K_FMT, V_FMT, 14, 0, kvarn=1, device=dev)
+    t_fill = fill(c, B, H, D, n, chunk=4096)
+    fill_bytes = B * H * n * (2 * D * 4 + ROW_K + ROW_V)
+    td = time_decode(c, B, Hq, D)
+    dbytes = B * H * n * (ROW_K + ROW_V) + 2 * B * Hq * D * 4
+    res["kvarn"] = {"decode_gbs": dbytes / td / 1e9, "decode_frac": dbytes / td / 1e9 / peak, "decode_us": td * 1e6,
+                    "append_fill_mtok_s": n * B / t_fill / 1e6, "append_fill_gbs": fill_bytes / t_fill / 1e9,
+                    "append_fill_frac": fill_bytes / t_fill / 1e9 / peak}
+    del c
+    torch.cuda.empty_cache()
+
+    # asymmetric low-bit sweep: batch 4, 4 kv heads, 65,536 positions, bf16 tail 1,024
+    B, H, Hq, D, n, W = 4, 4, 24, 256, 65536, 1024
+    sweep = {}
+    for kf, vf, name in [(5, 5, "q4_1/q4_1"), (5, 3, "q4_1/q3_1"), (3, 1, "q3_1/q2_1"), (0, 0, "q2_0/q2_0")]:
+        c = kvq.KVCache(1, B, H, Hq, D, n, kf, vf, 12, W, device=dev)
+        fill(c, B, H, D, n, outlier=False)
+        td = time_decode(c, B, Hq, D)
+        dbytes = B * H * ((n - W) * (rows_bytes(kf, D) + rows_bytes(vf, D)) + W * 2 * 512) + 2 * B * Hq * D * 4
+        sweep[name] = {"decode_gbs": dbytes / td / 1e9, "decode_frac": dbytes / td / 1e9 / peak}
+        del c
+        torch.cuda.empty_cache()
+    res["asymmetric_sweep"] = sweep
+    return res
 
 
 def main():
@@ -362,6 +491,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the large-workload figures")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -167,16 +167,13 @@ attn_pass1(P1Args a) {
 }
 
 // Merge of the split partials. One CTA per (b, row, q head) and 32-channel slice; its
-// 256 threads are 32 channels x 8 split groups. Weights e_s = 2^(m_s - M) go to shared
-// memory; group j sums splits j, j+8, j+16, ... in order and the 8 group sums are added
+// 256 threads are 32 channels x 8 split groups. Group j folds splits j, j+8, j+16, ... in
+// order with an online rescale (one pass over m, l and o), then the 8 groups are folded
 // in a fixed order, so the result is bit-reproducible.
 constexpr int MG = 8;
 __global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G,
                                                   int H, int D, int n_split) {
-    extern __shared__ float e[];               // [n_split] weights
-    __shared__ float red[MG][32];
-    __shared__ float wred[8];
-    __shared__ float Msh, Lsh;
+    __shared__ float sm_m[MG][32], sm_l[MG][32], sm_o[MG][32];
     const int hq = blockIdx.x % (G * H);
     const long long br = blockIdx.x / (G * H);
     const int h = hq / G, g = hq % G;
@@ -185,55 +182,39 @@ __global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, 
     const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
     asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the preceding pass(es)
 
-    float M = -INFINITY;
-    for (int s = tid; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * stride + g]);
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (lane == 0) wred[grp] = M;
-    __syncthreads();
-    if (tid == 0) {
-        float mm = -INFINITY;
-        for (int w = 0; w < MG; ++w) mm = fmaxf(mm, wred[w]);
-        Msh = mm;
-    }
-    __syncthreads();
-    M = Msh;
-    float lpart = 0.f;                         // fixed assignment: thread tid sums splits tid, tid+256, ...
-    for (int s = tid; s < n_split; s += blockDim.x) {
-        const float ms = base[s * stride + g];
-        const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-        e[s] = w;
-        lpart = fmaf(base[s * stride + G + g], w, lpart);
-    }
-    for (int off = 16; off >= 1; off >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, off);
-    __syncthreads();
-    if (lane == 0) wred[grp] = lpart;
-    __syncthreads();
-    if (tid == 0) {
-        float L = 0.f;
-        for (int w = 0; w < MG; ++w) L += wred[w];
-        Lsh = L;
-    }
     const int c = blockIdx.y * 32 + lane;
-    float acc = 0.f;
-    if (c < D) {
-        const float* ob = base + 2 * G + (long long)g * D + c;
-        int s = grp;
-        for (; s + 3 * MG < n_split; s += 4 * MG) {
-            const float o0 = ob[(long long)s * stride], o1 = ob[(long long)(s + MG) * stride];
-            const float o2 = ob[(long long)(s + 2 * MG) * stride], o3 = ob[(long long)(s + 3 * MG) * stride];
-            acc = fmaf(o0, e[s], acc);
-            acc = fmaf(o1, e[s + MG], acc);
-            acc = fmaf(o2, e[s + 2 * MG], acc);
-            acc = fmaf(o3, e[s + 3 * MG], acc);
+    const int cc = c < D ? c : D - 1;
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    for (int s = grp; s < n_split; s += MG) {
+        const float* ps = base + (long long)s * stride;
+        const float ms = ps[g], ls = ps[G + g], os = ps[2 * G + (long long)g * D + cc];
+        if (ms == -INFINITY) continue;
+        if (ms > M) {
+            const float e = (M == -INFINITY) ? 0.f : exp2f(M - ms);
+            L *= e;
+            O *= e;
+            M = ms;
         }
-        for (; s < n_split; s += MG) acc = fmaf(ob[(long long)s * stride], e[s], acc);
+        const float w = exp2f(ms - M);
+        L = fmaf(ls, w, L);
+        O = fmaf(os, w, O);
     }
-    red[grp][lane] = acc;
+    sm_m[grp][lane] = M;
+    sm_l[grp][lane] = L;
+    sm_o[grp][lane] = O;
     __syncthreads();
     if (grp == 0 && c < D) {
-        float O = 0.f;
-        for (int j = 0; j < MG; ++j) O += red[j][lane];
-        out[(br * H * G + hq) * (long long)D + c] = O / Lsh;
+        float Mt = -INFINITY;
+        for (int j = 0; j < MG; ++j) Mt = fmaxf(Mt, sm_m[j][lane]);
+        float Lt = 0.f, Ot = 0.f;
+        for (int j = 0; j < MG; ++j) {
+            const float mj = sm_m[j][lane];
+            if (mj == -INFINITY) continue;
+            const float w = exp2f(mj - Mt);
+            Lt = fmaf(sm_l[j][lane], w, Lt);
+            Ot = fmaf(sm_o[j][lane], w, Ot);
+        }
+        out[(br * H * G + hq) * (long long)D + c] = Ot / Lt;
     }
 }
 
@@ -265,7 +246,7 @@ SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int n
     chunk = (chunk + align - 1) / align * align;
     // ring rows run as a separate, later launch: cut them finer so it ends quickly
     long long rchunk = (n_ring + per_unit - 1) / per_unit;
-    if (rchunk < align) rchunk = align;
+    if (rchunk < 4 * align) rchunk = 4 * align;
     rchunk = (rchunk + align - 1) / align * align;
     p.main_chunk = chunk;
     p.ring_chunk = rchunk;
@@ -344,7 +325,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)lv.B * rows * lv.H * lv.G), (unsigned)((lv.D + 31) / 32));
     cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = (size_t)a.n_split * sizeof(float);
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -111,54 +111,15 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], CWARPS); }
-        *fault = 0;
-        fence_mbar_init();
-    }
     // Rows past the end of a partial tile are read (and multiplied by p = 0): zero the
     // stages once so such rows always hold finite values (stale rows of this region or 0).
     for (size_t i = threadIdx.x * 16; i < STAGES * sb; i += THREADS * 16)
         *reinterpret_cast<uint4*>(stage0 + i) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
-    // query fragments (B operand of QK, head g of lane (g, t)), shared by the consumer warps
-    if (warp == 0) {
-        const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
-#pragma unroll
-        for (int bb = 0; bb < NB; ++bb) {
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                float v[4];
-#pragma unroll
-                for (int sl = 0; sl < 4; ++sl) {
-                    const int c = 32 * bb + q_channel<KF>(t, m, sl);
-                    float x = (g < G) ? qg[c] * a.qscale : 0.f;
-                    if (kvarn) x *= sK[c];
-                    v[sl] = x;
-                }
-                uint32_t p01[3], p23[3];
-                split_pack<KF>(v[0], v[1], p01);
-                split_pack<KF>(v[2], v[3], p23);
-#pragma unroll
-                for (int pp = 0; pp < KP; ++pp) qs[((bb * 2 + m) * KP + pp) * 32 + lane] = make_uint2(p01[pp], p23[pp]);
-            }
-        }
-        if constexpr (KT::asym) {
-            // per-block sums of the (scaled) query channels, heads 0..7
-            for (int idx = lane; idx < NB * 8; idx += 32) {
-                const int bb = idx >> 3, hh = idx & 7;
-                float sacc = 0.f;
-                if (hh < G) {
-                    const float* qh = a.q + ((long long)br * G * H + (long long)h * G + hh) * D + 32 * bb;
-                    for (int c = 0; c < 32; ++c) {
-                        float x = qh[c] * a.qscale;
-                        if (kvarn) x *= sK[32 * bb + c];
-                        sacc += x;
-                    }
-                }
-                qsum_s[idx] = sacc;
-            }
-        }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], CWARPS); }
+        *fault = 0;
+        fence_mbar_init();
     }
     __syncthreads();
 
@@ -177,6 +138,53 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
                 bulk_g2s(st + (size_t)TOK * a.kstride, vreg + r0 * a.vstride, vb, &full[s]);
             }
         }
+    }
+
+    // ------------------------------------------------------------ query fragments
+    // (B operand of QK, head g of lane (g, t)), built while the first tiles are in flight:
+    // consumer warp w builds blocks w, w + 4 (and the asymmetric-format query sums),
+    // then the consumer warps meet at a named barrier.
+    if (warp < CWARPS) {
+        const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
+#pragma unroll
+        for (int bi = 0; bi < (NB + CWARPS - 1) / CWARPS; ++bi) {
+            const int bb = warp + CWARPS * bi;
+            if (bb < NB) {
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    float v[4];
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl) {
+                        const int c = 32 * bb + q_channel<KF>(t, m, sl);
+                        float x = (g < G) ? qg[c] * a.qscale : 0.f;
+                        if (kvarn) x *= sK[c];
+                        v[sl] = x;
+                    }
+                    uint32_t p01[3], p23[3];
+                    split_pack<KF>(v[0], v[1], p01);
+                    split_pack<KF>(v[2], v[3], p23);
+#pragma unroll
+                    for (int pp = 0; pp < KP; ++pp) qs[((bb * 2 + m) * KP + pp) * 32 + lane] = make_uint2(p01[pp], p23[pp]);
+                }
+            }
+        }
+        if constexpr (KT::asym) {
+            // per-block sums of the (scaled) query channels, heads 0..7
+            for (int idx = threadIdx.x; idx < NB * 8; idx += 32 * CWARPS) {
+                const int bb = idx >> 3, hh = idx & 7;
+                float sacc = 0.f;
+                if (hh < G) {
+                    const float* qh = a.q + ((long long)br * G * H + (long long)h * G + hh) * D + 32 * bb;
+                    for (int c = 0; c < 32; ++c) {
+                        float x = qh[c] * a.qscale;
+                        if (kvarn) x *= sK[32 * bb + c];
+                        sacc += x;
+                    }
+                }
+                qsum_s[idx] = sacc;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * CWARPS) : "memory");
     }
 
     // ------------------------------------------------------------ consumers
