@@ -32,6 +32,30 @@ struct Lanes {
     static constexpr int LPB = 32 / CPL;   // lanes per 32-value block
 };
 
+// rhaz(fl(x / d)) for d > 0 without a division in the common case: r = x * fl(1/d) is
+// within 1.5 * 2^-23 relative of fl(x / d); unless r lies within 4e-7 * |r| of a half-integer,
+// both round to the same integer. Near a half-integer the true IEEE quotient decides.
+__device__ __forceinline__ float rhaz_div(float x, float d, float rd) {
+    float r = __fmul_rn(x, rd);
+    const float ar = fabsf(r);
+    const float fr = ar - floorf(ar);
+    if (fabsf(fr - 0.5f) <= 4e-7f * ar) r = __fdiv_rn(x, d);
+    return roundf(r);
+}
+
+// pack CPL codes (bits below W0 into plane 0, the next W1 bits into plane 1) and store
+template <int CPL, int W0, int W1>
+__device__ __forceinline__ void pack_store(uint8_t* p0, uint8_t* p1, int lane, const uint32_t (&u)[CPL]) {
+    uint64_t v0 = 0, v1 = 0;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        v0 |= (uint64_t)(u[j] & ((1u << W0) - 1)) << (j * W0);
+        if constexpr (W1 > 0) v1 |= (uint64_t)(u[j] >> W0) << (j * W1);
+    }
+    store_plane_bits(p0, lane, CPL * W0, v0);
+    if constexpr (W1 > 0) store_plane_bits(p1, lane, CPL * W1, v1);
+}
+
 // Quantize this lane's CPL values into row `row` of format f (all lanes participate).
 template <int CPL>
 __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFmt& f, int lane,
@@ -67,11 +91,13 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         const float d32 = __fdiv_rn(a, (float)qmax);
         dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
+        const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
             float r = 0.f;
-            if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(x[j], d)), (float)-qmax), (float)qmax);
-            u[j] = (uint32_t)((int)r + qmax + 1);
+            if (d != 0.f) r = fminf(fmaxf(rhaz_div(x[j], d, rd), (float)-qmax), (float)qmax);
+            // exact float -> int through the 1.5 * 2^23 magic (|r| <= 127)
+            u[j] = (uint32_t)(__float_as_int(r + 12582912.0f) - 0x4B400000 + qmax + 1);
         }
     } else {
         const int umax = (1 << f.bits) - 1;
@@ -85,22 +111,24 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
         const float m = __half2float(__ushort_as_half(mh));
+        const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
             float r = 0.f;
-            if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(__fsub_rn(x[j], m), d)), 0.f), (float)umax);
-            u[j] = (uint32_t)r;
+            if (d != 0.f) r = fminf(fmaxf(rhaz_div(__fsub_rn(x[j], m), d, rd), 0.f), (float)umax);
+            u[j] = (uint32_t)(__float_as_int(r + 12582912.0f) - 0x4B400000);
         }
     }
-    uint64_t v0 = 0, v1 = 0;
-    const uint32_t m0 = (1u << f.w0) - 1;
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-        v0 |= (uint64_t)(u[j] & m0) << (j * f.w0);
-        if (f.w1) v1 |= (uint64_t)(u[j] >> f.w0) << (j * f.w1);
+    uint8_t* p0 = row + f.off_p0;
+    uint8_t* p1 = row + f.off_p1;
+    switch (f.bits) {
+        case 8: pack_store<CPL, 8, 0>(p0, p1, lane, u); break;
+        case 6: pack_store<CPL, 4, 2>(p0, p1, lane, u); break;
+        case 5: pack_store<CPL, 4, 1>(p0, p1, lane, u); break;
+        case 4: pack_store<CPL, 4, 0>(p0, p1, lane, u); break;
+        case 3: pack_store<CPL, 2, 1>(p0, p1, lane, u); break;
+        default: pack_store<CPL, 2, 0>(p0, p1, lane, u); break;
     }
-    store_plane_bits(row + f.off_p0, lane, CPL * f.w0, v0);
-    if (f.w1) store_plane_bits(row + f.off_p1, lane, CPL * f.w1, v1);
     if ((lane % LPB) == 0) {
         reinterpret_cast<uint16_t*>(row)[blk] = dh;
         if (f.asym) reinterpret_cast<uint16_t*>(row + f.off_m)[blk] = mh;
@@ -165,10 +193,11 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
             a = group_max<LPB>(a);
             const float d32 = __fdiv_rn(a, 127.f);
             const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
+            const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
 #pragma unroll
             for (int j = 0; j < CPL; ++j) {
                 float r = 0.f;
-                if (d != 0.f) r = fminf(fmaxf(roundf(__fdiv_rn(x[j], d)), -127.f), 127.f);
+                if (d != 0.f) r = fminf(fmaxf(rhaz_div(x[j], d, rd), -127.f), 127.f);
                 t[j] = __fmul_rn(d, r);
             }
         }

@@ -246,7 +246,7 @@ SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int n
     chunk = (chunk + align - 1) / align * align;
     // ring rows run as a separate, later launch: cut them finer so it ends quickly
     long long rchunk = (n_ring + per_unit - 1) / per_unit;
-    if (rchunk < 4 * align) rchunk = 4 * align;
+    if (rchunk < align) rchunk = align;
     rchunk = (rchunk + align - 1) / align * align;
     p.main_chunk = chunk;
     p.ring_chunk = rchunk;

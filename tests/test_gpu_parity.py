@@ -177,3 +177,39 @@ def test_prefill_formats(D, tail, W):
         out = g.prefill(0, to_dev(q), 0.75).cpu().numpy()
         ref = o.prefill(0, q, 0.75)
         check_close(out, ref, vmax, f"prefill kf={kf} vf={vf} tail={tail} W={W} D={D} kvarn={kvarn}")
+
+
+@pytest.mark.parametrize("tail,W", [(orc.NONE, 0), (orc.Q8_0, 8)])
+def test_append_half_step_ties(tail, W):
+    """Values placed exactly on code half-steps (x / d = k + 1/2, and (x - m) / d = k + 1/2
+    for qX_1): the quantizer must round them away from zero exactly as the oracle's IEEE
+    division does, for every format (the kernel's division-free path falls back to a true
+    division next to half-steps)."""
+    import torch
+    from quantized_mixed_precision_qx_b200.kvq import KVCache
+    rng = np.random.default_rng(77)
+    T, H, D = 40, 1, 64
+    for f in range(12):
+        X = orc.fmt_bits(f)
+        d = np.float32(2.0 ** -5)
+        x = np.empty((1, T, H, D), np.float32)
+        for t in range(T):
+            for blk in range(D // 32):
+                if orc.fmt_asym(f):
+                    umax = (1 << X) - 1
+                    m = np.float32(-0.375)
+                    k = rng.integers(0, umax, 32).astype(np.float32)
+                    vals = m + (k + np.float32(0.5)) * d
+                    vals[0] = m                       # min -> m exactly
+                    vals[1] = m + umax * d            # max -> d = (max - min) / umax exactly
+                else:
+                    qmax = (1 << (X - 1)) - 1
+                    k = rng.integers(-qmax, qmax, 32).astype(np.float32)
+                    vals = (k + np.float32(0.5)) * d
+                    vals[0] = qmax * d                # absmax -> d exactly
+                x[0, t, 0, 32 * blk:32 * blk + 32] = vals.astype(np.float32)
+        g = KVCache(1, 1, H, 2, D, T, f, f, tail, W)
+        o = orc.Cache(1, 1, H, 2, D, T, f, f, tail, W)
+        g.append(0, torch.from_numpy(x).cuda(), torch.from_numpy(x).cuda())
+        o.append(0, x, x)
+        compare_bytes(g, o, 0, 1, H, T, W)
