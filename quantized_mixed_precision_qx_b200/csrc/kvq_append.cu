@@ -36,11 +36,12 @@ struct Lanes {
 // within 1.5 * 2^-23 relative of fl(x / d); unless r lies within 4e-7 * |r| of a half-integer,
 // both round to the same integer. Near a half-integer the true IEEE quotient decides.
 __device__ __forceinline__ float rhaz_div(float x, float d, float rd) {
-    float r = __fmul_rn(x, rd);
+    const float r = __fmul_rn(x, rd);
     const float ar = fabsf(r);
-    const float fr = ar - floorf(ar);
-    if (fabsf(fr - 0.5f) <= 4e-7f * ar) r = __fdiv_rn(x, d);
-    return roundf(r);
+    const float fl = floorf(ar);
+    const float fr = ar - fl;                        // exact
+    if (fabsf(fr - 0.5f) <= 4e-7f * ar) return roundf(__fdiv_rn(x, d));
+    return copysignf(fr > 0.5f ? fl + 1.f : fl, r);  // nearest integer, away from the half point
 }
 
 // pack CPL codes (bits below W0 into plane 0, the next W1 bits into plane 1) and store
