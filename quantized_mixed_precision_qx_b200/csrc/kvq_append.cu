@@ -32,16 +32,37 @@ struct Lanes {
     static constexpr int LPB = 32 / CPL;   // lanes per 32-value block
 };
 
-// rhaz(fl(x / d)) for d > 0 without a division in the common case: r = x * fl(1/d) is
-// within 1.5 * 2^-23 relative of fl(x / d); unless r lies within 4e-7 * |r| of a half-integer,
-// both round to the same integer. Near a half-integer the true IEEE quotient decides.
-__device__ __forceinline__ float rhaz_div(float x, float d, float rd) {
-    const float r = __fmul_rn(x, rd);
-    const float ar = fabsf(r);
-    const float fl = floorf(ar);
-    const float fr = ar - fl;                        // exact
-    if (fabsf(fr - 0.5f) <= 4e-7f * ar) return roundf(__fdiv_rn(x, d));
-    return copysignf(fr > 0.5f ? fl + 1.f : fl, r);  // nearest integer, away from the half point
+constexpr float MAGIC = 12582912.0f;          // 1.5 * 2^23: adding it rounds |r| < 2^22 to an integer
+constexpr int MAGIC_BITS = 0x4B400000;         // bit pattern of MAGIC
+
+// Codes rhaz(fl((x_j - m) / d)) clamped to [lo, hi], for d > 0 (all zero when d == 0), returned as
+// t_j = MAGIC + code (so code = bits(t_j) - MAGIC_BITS and the code as a float is t_j - MAGIC).
+// r = (x - m) * fl(1/d) is within 1.5 * 2^-23 * |r| of fl((x - m) / d). Clamping to integer bounds
+// commutes with rounding, and after it |r| <= lim = max(|lo|, |hi|), so unless r lies within
+// 4e-7 * lim of a half-integer both have the same nearest integer (which is then not a tie) and
+// the rounding add gives it. A lane with such a near-tie redoes its values from the correctly
+// rounded IEEE quotient, once for all CPL values.
+template <int CPL, bool ASYM>
+__device__ __forceinline__ void round_codes(const float (&x)[CPL], float d, float m, float lo, float hi,
+                                            float (&t)[CPL]) {
+    const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
+    const float tol = 4e-7f * fmaxf(-lo, hi);
+    bool near = false;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const float v = ASYM ? __fsub_rn(x[j], m) : x[j];
+        const float r = fminf(fmaxf(__fmul_rn(v, rd), lo), hi);
+        t[j] = __fadd_rn(r, MAGIC);
+        const float e = __fsub_rn(r, __fsub_rn(t[j], MAGIC));     // exact, |e| <= 1/2
+        near |= fabsf(__fsub_rn(fabsf(e), 0.5f)) <= tol;
+    }
+    if (near) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const float v = ASYM ? __fsub_rn(x[j], m) : x[j];
+            t[j] = __fadd_rn(fminf(fmaxf(roundf(__fdiv_rn(v, d)), lo), hi), MAGIC);
+        }
+    }
 }
 
 // pack CPL codes (bits below W0 into plane 0, the next W1 bits into plane 1) and store
@@ -92,14 +113,10 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         const float d32 = __fdiv_rn(a, (float)qmax);
         dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
-        const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
+        float t[CPL];
+        round_codes<CPL, false>(x, d, 0.f, (float)-qmax, (float)qmax, t);
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-            float r = 0.f;
-            if (d != 0.f) r = fminf(fmaxf(rhaz_div(x[j], d, rd), (float)-qmax), (float)qmax);
-            // exact float -> int through the 1.5 * 2^23 magic (|r| <= 127)
-            u[j] = (uint32_t)(__float_as_int(r + 12582912.0f) - 0x4B400000 + qmax + 1);
-        }
+        for (int j = 0; j < CPL; ++j) u[j] = (uint32_t)(__float_as_int(t[j]) - (MAGIC_BITS - qmax - 1));
     } else {
         const int umax = (1 << f.bits) - 1;
         float lo = x[0], hi = x[0];
@@ -112,13 +129,10 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
         const float m = __half2float(__ushort_as_half(mh));
-        const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
+        float t[CPL];
+        round_codes<CPL, true>(x, d, m, 0.f, (float)umax, t);
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-            float r = 0.f;
-            if (d != 0.f) r = fminf(fmaxf(rhaz_div(__fsub_rn(x[j], m), d, rd), 0.f), (float)umax);
-            u[j] = (uint32_t)(__float_as_int(r + 12582912.0f) - 0x4B400000);
-        }
+        for (int j = 0; j < CPL; ++j) u[j] = (uint32_t)(__float_as_int(t[j]) - MAGIC_BITS);
     }
     uint8_t* p0 = row + f.off_p0;
     uint8_t* p1 = row + f.off_p1;
@@ -149,33 +163,34 @@ __device__ __forceinline__ void store_low(uint8_t* row, const RowFmt& f, const f
 
 template <int CPL>
 __global__ void __launch_bounds__(32 * WARPS_PER_CTA)
-append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, long long n, int C) {
+append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C) {
     const int lane = threadIdx.x & 31;
-    const long long item = (long long)blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-    const long long items = (long long)C * lv.B * lv.H * 2;
-    if (item >= items) return;
-    // item order: (b, i, h, kv) so consecutive warps read consecutive input rows
-    const int kv = (int)(item & 1);
-    const int h = (int)((item >> 1) % lv.H);
-    const long long bi = (item >> 1) / lv.H;
-    const int i = (int)(bi % C);
-    const int b = (int)(bi / C);
+    // item order: (b, i, h, kv) so consecutive warps read consecutive input rows; the host
+    // keeps C * B * H * 2 below 2^32 and positions below 2^31
+    const uint32_t item = blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+    const uint32_t per_pos = 2u * (uint32_t)lv.H;
+    const uint32_t row = item / per_pos;                 // b * C + i
+    if (row >= C * (uint32_t)lv.B) return;
+    const uint32_t kv = item & 1u;
+    const uint32_t h = (item - row * per_pos) >> 1;
+    const uint32_t b = row / C;
+    const uint32_t i = row - b * C;
     const int D = lv.D;
-    const float* src = (kv ? v : k) + (((long long)b * C + i) * lv.H + h) * D;
+    const float* src = (kv ? v : k) + ((long long)row * lv.H + h) * D;
     const RowFmt fl = kv ? lv.fmt[1] : lv.fmt[0];   // by value: no pointer into the parameters
     uint8_t* main = lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv];
     const float* s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * D : nullptr;
-    const long long p = n + i;
+    const uint32_t p = n + i;
 
     float x[CPL];
     load_row_f32<CPL>(src, lane, x);
 
     if (lv.W == 0) {
-        store_low<CPL>(main + p * fl.stride, fl, s, lane, x);
+        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, x);
         return;
     }
-    const long long W = lv.W;
-    if (p < n + C - W) {
+    const uint32_t W = (uint32_t)lv.W;
+    if (i + W < C) {
         // enters and leaves the window inside this append: tail rounding, then low-bit
         float t[CPL];
         // round through the tail format in registers (same values a ring round trip gives)
@@ -194,28 +209,26 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
             a = group_max<LPB>(a);
             const float d32 = __fdiv_rn(a, 127.f);
             const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
-            const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
+            float c[CPL];
+            round_codes<CPL, false>(x, d, 0.f, -127.f, 127.f, c);
 #pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                float r = 0.f;
-                if (d != 0.f) r = fminf(fmaxf(rhaz_div(x[j], d, rd), -127.f), 127.f);
-                t[j] = __fmul_rn(d, r);
-            }
+            for (int j = 0; j < CPL; ++j) t[j] = __fmul_rn(d, __fsub_rn(c[j], MAGIC));
         }
-        store_low<CPL>(main + p * fl.stride, fl, s, lane, t);
+        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, t);
         return;
     }
     // ends inside the window: evict the slot's old occupant, then take the slot
     uint8_t* ring = lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region;
-    const long long slot = p % W;
-    uint8_t* srow = ring + slot * lv.tail.stride;
-    const long long base = n - W;                       // old window start (may be < 0)
-    const long long q = base + ((slot - base) % W + W) % W;
+    const uint32_t im = i % W;
+    const uint32_t slot = (n % W + im) % W;
+    uint8_t* srow = ring + (long long)slot * lv.tail.stride;
+    // old occupant: the position in [n - W, n) congruent to p = n + i modulo W
+    const long long q = (long long)n - W + im;
     if (q >= 0) {
         float y[CPL];
         load_row_values<CPL>(srow, lv.tail, lane, y);
         __syncwarp();
-        store_low<CPL>(main + q * fl.stride, fl, s, lane, y);
+        store_low<CPL>(main + (long long)q * fl.stride, fl, s, lane, y);
     }
     __syncwarp();
     store_row<CPL>(srow, lv.tail, lane, x);
@@ -262,13 +275,15 @@ __global__ void calibrate_kernel(LayerView lv, const float* __restrict__ k, cons
 cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
                           cudaStream_t st) {
     const long long items = (long long)C * lv.B * lv.H * 2;
+    if (items >= (1LL << 32) - WARPS_PER_CTA || n + C > (1LL << 31)) return cudaErrorInvalidValue;
     const unsigned grid = (unsigned)((items + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
     const dim3 block(32 * WARPS_PER_CTA);
+    const uint32_t n32 = (uint32_t)n, C32 = (uint32_t)C;
     switch (lv.D / 32) {
-        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
-        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
-        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
-        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n, C); break;
+        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
+        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
+        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
+        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

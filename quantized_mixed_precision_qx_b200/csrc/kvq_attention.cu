@@ -170,8 +170,10 @@ attn_pass1(P1Args a) {
 // 256 threads are 32 channels x 8 split groups. Group j folds splits j, j+8, j+16, ... in
 // order with an online rescale (one pass over m, l and o), then the 8 groups are folded
 // in a fixed order, so the result is bit-reproducible.
-constexpr int MG = 8;
-__global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G,
+constexpr int MG = 16;
+constexpr int MU = 4;   // partials per merge step
+
+__global__ void __launch_bounds__(32 * MG) attn_merge(const float* __restrict__ ws, float* __restrict__ out, int G,
                                                   int H, int D, int n_split) {
     __shared__ float sm_m[MG][32], sm_l[MG][32], sm_o[MG][32];
     const int hq = blockIdx.x % (G * H);
@@ -185,19 +187,36 @@ __global__ void __launch_bounds__(256) attn_merge(const float* __restrict__ ws, 
     const int c = blockIdx.y * 32 + lane;
     const int cc = c < D ? c : D - 1;
     float M = -INFINITY, L = 0.f, O = 0.f;
-    for (int s = grp; s < n_split; s += MG) {
-        const float* ps = base + (long long)s * stride;
-        const float ms = ps[g], ls = ps[G + g], os = ps[2 * G + (long long)g * D + cc];
-        if (ms == -INFINITY) continue;
-        if (ms > M) {
-            const float e = (M == -INFINITY) ? 0.f : exp2f(M - ms);
+    // MU partials per step: their loads are independent and in flight together; one rescale
+    // of the running sums per step
+    for (int s0 = grp; s0 < n_split; s0 += MG * MU) {
+        float ms[MU], ls[MU], os[MU];
+#pragma unroll
+        for (int u = 0; u < MU; ++u) {
+            const int s = s0 + u * MG;
+            ms[u] = -INFINITY; ls[u] = 0.f; os[u] = 0.f;
+            if (s < n_split) {
+                const float* ps = base + (long long)s * stride;
+                ms[u] = ps[g]; ls[u] = ps[G + g]; os[u] = ps[2 * G + (long long)g * D + cc];
+            }
+        }
+        float mx = M;
+#pragma unroll
+        for (int u = 0; u < MU; ++u) mx = fmaxf(mx, ms[u]);
+        if (mx == -INFINITY) continue;
+        if (mx > M) {
+            const float e = (M == -INFINITY) ? 0.f : exp2f(M - mx);
             L *= e;
             O *= e;
-            M = ms;
+            M = mx;
         }
-        const float w = exp2f(ms - M);
-        L = fmaf(ls, w, L);
-        O = fmaf(os, w, O);
+#pragma unroll
+        for (int u = 0; u < MU; ++u) {
+            if (ms[u] == -INFINITY) continue;
+            const float w = exp2f(ms[u] - M);
+            L = fmaf(ls[u], w, L);
+            O = fmaf(os[u], w, O);
+        }
     }
     sm_m[grp][lane] = M;
     sm_l[grp][lane] = L;
@@ -235,23 +254,33 @@ bool use_tensor_cores(int D) { return D == 128 || D == 256; }
 
 SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, bool tc) {
     SplitPlan p{};
-    const long long total = n_main + n_ring;
     const long long target = (tc ? 3LL : 4LL) * num_sms;
     long long per_unit = (target + units - 1) / units;
     if (per_unit < 1) per_unit = 1;
-    const long long align = tc ? tc::TOK : 16;
-    // low-bit rows: about per_unit splits of at least 4 tiles each
-    long long chunk = (n_main + per_unit - 1) / per_unit;
-    if (chunk < 4 * align) chunk = 4 * align;
-    chunk = (chunk + align - 1) / align * align;
-    // ring rows run as a separate, later launch: cut them finer so it ends quickly
+    if (tc) {
+        // every split of either region gets the same number of tiles, chosen so that both
+        // regions' splits fit in about one wave (per_unit per unit, 3 CTAs per SM): the ring
+        // pass and the low-bit pass then run side by side and end together
+        const long long tr = (n_ring + tc::TOK - 1) / tc::TOK, tm = (n_main + tc::TOK - 1) / tc::TOK;
+        long long per = (tr + tm + per_unit - 1) / per_unit;
+        if (per < 1) per = 1;
+        p.ring_chunk = p.main_chunk = per * tc::TOK;
+        p.n_ring_split = (int)((tr + per - 1) / per);
+        p.n_main_split = (int)((tm + per - 1) / per);
+        return p;
+    }
+    // CUDA-core path: about per_unit splits per region, low-bit splits of at least 64 rows
+    const long long align = 16;
     long long rchunk = (n_ring + per_unit - 1) / per_unit;
     if (rchunk < align) rchunk = align;
     rchunk = (rchunk + align - 1) / align * align;
-    p.main_chunk = chunk;
+    long long chunk = (n_main + per_unit - 1) / per_unit;
+    if (chunk < 4 * align) chunk = 4 * align;
+    chunk = (chunk + align - 1) / align * align;
     p.ring_chunk = rchunk;
-    p.n_main_split = (int)((n_main + chunk - 1) / chunk);
+    p.main_chunk = chunk;
     p.n_ring_split = (int)((n_ring + rchunk - 1) / rchunk);
+    p.n_main_split = (int)((n_main + chunk - 1) / chunk);
     return p;
 }
 
@@ -272,7 +301,10 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     const int CPL = lv.D / 32;
     const bool tcp = use_tensor_cores(lv.D);
     int launched = 0;
-    for (int region = 0; region < 2; ++region) {
+    // the ring pass goes first: its few short splits take their SM slots before the
+    // low-bit pass fills the rest, instead of waiting for low-bit splits to retire
+    for (int ri = 0; ri < 2; ++ri) {
+        const int region = 1 - ri;
         a.ring = region;
         a.chunk = region ? plan.ring_chunk : plan.main_chunk;
         a.region_rows = region ? n_ring : n_main;
@@ -324,7 +356,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     // the merge is a programmatic dependent: it launches early and waits for the passes
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((long long)lv.B * rows * lv.H * lv.G), (unsigned)((lv.D + 31) / 32));
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(32 * MG);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

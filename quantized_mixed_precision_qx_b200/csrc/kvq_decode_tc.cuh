@@ -56,7 +56,7 @@ struct Args {
 __host__ __device__ constexpr size_t stage_bytes(int ks, int vs) { return (size_t)TOK * (ks + vs); }
 // shared memory: [stages | final combine (aliased)] [P transpose] [mbarriers] [fault word]
 __host__ __device__ constexpr size_t comb_bytes(int D) {
-    return (size_t)(CWARPS * 8 * 2 + CWARPS * 8 * NBMAX + CWARPS * 8 * D) * sizeof(float);
+    return (size_t)(CWARPS * 8 * 3 + 16 + CWARPS * 8 * NBMAX + CWARPS * 8 * D) * sizeof(float);
 }
 __host__ __device__ constexpr size_t main_bytes(int ks, int vs, int D) {
     return ((STAGES * stage_bytes(ks, vs) > comb_bytes(D) ? STAGES * stage_bytes(ks, vs) : comb_bytes(D)) + 127) & ~(size_t)127;
@@ -111,10 +111,37 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // Rows past the end of a partial tile are read (and multiplied by p = 0): zero the
-    // stages once so such rows always hold finite values (stale rows of this region or 0).
-    for (size_t i = threadIdx.x * 16; i < STAGES * sb; i += THREADS * 16)
-        *reinterpret_cast<uint4*>(stage0 + i) = make_uint4(0, 0, 0, 0);
+    // query values of this lane's fragments, loaded first so their latency overlaps the setup
+    constexpr int QB = (NB + CWARPS - 1) / CWARPS;
+    float qv[QB][2][4];
+    if (warp < CWARPS) {
+        const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
+#pragma unroll
+        for (int bi = 0; bi < QB; ++bi) {
+            const int bb = warp + CWARPS * bi;
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const int c = 32 * bb + q_channel<KF>(t, m, sl);
+                    qv[bi][m][sl] = (bb < NB && g < G) ? qg[c] : 0.f;
+                }
+        }
+    }
+    // Rows past the end of a partial last tile are read (and multiplied by p = 0): zero
+    // them in that tile's stage so they always hold finite values.
+    if (n_tiles > 0) {
+        const int last_rows = (int)(t1 - t0 - (long long)(n_tiles - 1) * TOK);
+        if (last_rows < TOK) {
+            uint8_t* st = stage0 + ((n_tiles - 1) % STAGES) * sb;
+            const int kz0 = last_rows * a.kstride, kz1 = TOK * a.kstride;
+            const int vz0 = kz1 + last_rows * a.vstride, vz1 = kz1 + TOK * a.vstride;
+            for (int i = kz0 + threadIdx.x * 16; i < kz1; i += THREADS * 16)
+                *reinterpret_cast<uint4*>(st + i) = make_uint4(0, 0, 0, 0);
+            for (int i = vz0 + threadIdx.x * 16; i < vz1; i += THREADS * 16)
+                *reinterpret_cast<uint4*>(st + i) = make_uint4(0, 0, 0, 0);
+        }
+    }
     fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], CWARPS); }
@@ -145,9 +172,8 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     // consumer warp w builds blocks w, w + 4 (and the asymmetric-format query sums),
     // then the consumer warps meet at a named barrier.
     if (warp < CWARPS) {
-        const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
 #pragma unroll
-        for (int bi = 0; bi < (NB + CWARPS - 1) / CWARPS; ++bi) {
+        for (int bi = 0; bi < QB; ++bi) {
             const int bb = warp + CWARPS * bi;
             if (bb < NB) {
 #pragma unroll
@@ -155,9 +181,8 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
                     float v[4];
 #pragma unroll
                     for (int sl = 0; sl < 4; ++sl) {
-                        const int c = 32 * bb + q_channel<KF>(t, m, sl);
-                        float x = (g < G) ? qg[c] * a.qscale : 0.f;
-                        if (kvarn) x *= sK[c];
+                        float x = qv[bi][m][sl] * a.qscale;
+                        if (kvarn) x *= sK[32 * bb + q_channel<KF>(t, m, sl)];
                         v[sl] = x;
                     }
                     uint32_t p01[3], p23[3];
@@ -408,31 +433,51 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
             }
         }
     }
-    __syncthreads();
-    float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
+    // per head: max over the warps, each warp's weight and the weighted sum of l
+    float* cw = co + CWARPS * 8 * D;      // [CWARPS][8]
+    float* cM = cw + CWARPS * 8;          // [8]
+    float* cL = cM + 8;                   // [8]
     const bool bad = *fault != 0;
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int hh = idx / D, c = idx % D;
+    if (threadIdx.x < 8) {
+        const int hh = threadIdx.x;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, cm[w * 8 + hh]);
-        float O = 0.f, L = 0.f;
-        if (M != -INFINITY) {
+        float L = 0.f;
 #pragma unroll
-            for (int w = 0; w < CWARPS; ++w) {
-                const float mw = cm[w * 8 + hh];
-                if (mw == -INFINITY) continue;
-                const float e = ex2(mw - M);
-                float ow = co[(w * 8 + hh) * D + c];
-                if constexpr (VT::asym) ow += cpm[(w * 8 + hh) * NBMAX + (c >> 5)];
-                O = fmaf(ow, e, O);
-                L = fmaf(cl[w * 8 + hh], e, L);
-            }
+        for (int w = 0; w < CWARPS; ++w) {
+            const float mw = cm[w * 8 + hh];
+            const float e = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2(mw - M);
+            cw[w * 8 + hh] = e;
+            L = fmaf(cl[w * 8 + hh], e, L);
         }
-        if (sV) O *= sV[c];
-        if (bad) L = __int_as_float(0x7fc00000);   // a timed-out wait poisons the result
-        part[2 * G + idx] = O;
-        if (c == 0) { part[hh] = M; part[G + hh] = L; }
+        cM[hh] = M;
+        cL[hh] = bad ? __int_as_float(0x7fc00000) : L;   // a timed-out wait poisons the result
+    }
+    __syncthreads();
+    float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
+    // o = sum over warps of weight * o_w, two channels per thread step (8-byte stores)
+    for (int idx = 2 * threadIdx.x; idx < G * D; idx += 2 * THREADS) {
+        const int hh = idx / D, c = idx % D;
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < CWARPS; ++w) {
+            const float e = cw[w * 8 + hh];
+            float2 ow = *reinterpret_cast<const float2*>(&co[(w * 8 + hh) * D + c]);
+            if constexpr (VT::asym) {
+                const float pmw = cpm[(w * 8 + hh) * NBMAX + (c >> 5)];
+                ow.x += pmw;
+                ow.y += pmw;
+            }
+            o0 = fmaf(ow.x, e, o0);
+            o1 = fmaf(ow.y, e, o1);
+        }
+        if (sV) { o0 *= sV[c]; o1 *= sV[c + 1]; }
+        *reinterpret_cast<float2*>(&part[2 * G + idx]) = make_float2(o0, o1);
+    }
+    if (threadIdx.x < G) {
+        part[threadIdx.x] = cM[threadIdx.x];
+        part[G + threadIdx.x] = cL[threadIdx.x];
     }
     if (a.dependent) asm volatile("griddepcontrol.wait;" ::: "memory");
 }

@@ -226,6 +226,13 @@ __device__ __forceinline__ void kperm8(const float (&x)[8], float (&y)[8]) {
     y[0] = x[0]; y[1] = x[4]; y[2] = x[1]; y[3] = x[5]; y[4] = x[2]; y[5] = x[6]; y[6] = x[3]; y[7] = x[7];
 }
 
+// Position order inside a 64-position tile: K~ row r, S / P column r and V~^T k-slot r all hold
+// position t0 + slot_pos(r), the 8 x 8 transpose of the natural order. A thread that fills k-slots
+// 8m .. 8m+7 of V~^T then reads staged rows m, m+8, .., m+56, so the 8 lanes with consecutive m
+// read consecutive rows (row strides are 16-byte multiples, so rows 8 apart share banks).
+__host__ __device__ constexpr int slot_pos(int r) { return ((r & 7) << 3) | (r >> 3); }
+static_assert(PN == 64, "slot_pos is the 8 x 8 transpose of a 64-position tile");
+
 // Staging of one tile's raw rows (K rows then V rows), filled by bulk copies: positions
 // below the window come from the low-bit store, the others from the ring (in position
 // order, the ring slot range split at its wrap).
@@ -412,7 +419,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 const int u = tid + i * PTHREADS;
                 const int kr = u / CHUNKS, ch = u % CHUNKS;
                 uint32_t sel;
-                const uint8_t* row = srow(0, t0, t0 + kr, sel);
+                const uint8_t* row = srow(0, t0, t0 + slot_pos(kr), sel);
                 uint32_t out[8];
                 if (kmode != 0) {
                     const int cb = ch >> 2, ct = ch & 3;
@@ -475,7 +482,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                     const uint8_t* rr[8];
                     uint32_t sel;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) rr[j] = srow(1, t0, t0 + 8 * pg + j, sel);
+                    for (int j = 0; j < 8; ++j) rr[j] = srow(1, t0, t0 + pg + 8 * j, sel);
                     uint32_t o[4][8];
                     switch (vfid) {
                         case F_Q2_0: v_chunk_fast<F_Q2_0, NB>(rr, vb, g, o); break;
@@ -497,7 +504,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             if (cc < CHUNKS) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int t = t0 + 8 * tg + j;
+                    const int t = t0 + tg + 8 * j;
                     uint32_t sel;
                     const uint8_t* row = srow(1, t0, t, sel);
                     Raw8 rv;
@@ -555,7 +562,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 t5::tmem_ld32(t_s + lane_off + hc, sv);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float v = (!full && t0 + hc + i > my_limit) ? -INFINITY : sv[i];
+                    const float v = (!full && t0 + slot_pos(hc + i) > my_limit) ? -INFINITY : sv[i];
                     mx = fmaxf(mx, v);
                 }
             }
@@ -584,7 +591,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 t5::tmem_ld32(t_s + lane_off + hc, sv);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool vis = full || t0 + hc + i <= my_limit;
+                    const bool vis = full || t0 + slot_pos(hc + i) <= my_limit;
                     const float p = (m_run == -INFINITY || !vis) ? 0.f : mma::ex2(sv[i] - m_run);
                     sv[i] = p;
                     ps += p;

@@ -3,6 +3,10 @@
     python -m quantized_mixed_precision_qx_b200.perf decode  --n 131072 [shape/format options]
     python -m quantized_mixed_precision_qx_b200.perf prefill --n 32768 --chunk 1024
     python -m quantized_mixed_precision_qx_b200.perf append  --n 65536 --chunk 8192
+    python -m quantized_mixed_precision_qx_b200.perf sweep   --n 32768 --step 1024
+
+`sweep` fills the cache by appends of --step positions and times one decode after each
+(the decode-after-append pattern of a generation loop), printing one JSON line per context.
 
 The cache is filled with seeded device-generated inputs (K ~ N(0,1) with 8 channels per head
 scaled x8, V ~ N(0,1)); the measured call is repeated --reps times (the first --warmup calls
@@ -25,7 +29,7 @@ def main():
     from quantized_mixed_precision_qx_b200 import kvq
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["decode", "prefill", "append"])
+    ap.add_argument("op", choices=["decode", "prefill", "append", "sweep"])
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--H", type=int, default=4)
     ap.add_argument("--Hq", type=int, default=24)
@@ -39,6 +43,9 @@ def main():
     ap.add_argument("--kvarn", type=int, default=0)
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--step", type=int, default=1024, help="sweep: positions appended between decodes")
+    ap.add_argument("--clean-flush", type=int, default=0,
+                    help="after the 256 MB flush write, read another 256 MB so L2 holds clean lines")
     a = ap.parse_args()
     dev = torch.device("cuda")
     kf, vf, tf = FMTS[a.k], FMTS[a.v], FMTS[a.tail]
@@ -57,6 +64,9 @@ def main():
         return (torch.randn(a.B, rows, a.H, a.D, device=dev, generator=gen) * scale,
                 torch.randn(a.B, rows, a.H, a.D, device=dev, generator=gen))
 
+    if a.op == "sweep":
+        sweep(a, c, kv, kf, vf, tf, W, dev, gen)
+        return
     t = 0
     while t < a.n:
         cc = min(8192, a.n - t)
@@ -121,6 +131,45 @@ def main():
         tm = statistics.median(times)
         res.update(us=tm * 1e6, mtok_s=a.chunk * a.B / tm / 1e6)
     print(json.dumps(res), flush=True)
+
+
+def decode_bytes(a, n, kf, vf, tf, W):
+    rk, rv = BLOCK_BYTES[kf] * a.D // 32, BLOCK_BYTES[vf] * a.D // 32
+    rt = BLOCK_BYTES.get(tf, 0) * a.D // 32
+    ring = min(n, W)
+    return a.B * a.H * ((n - ring) * (rk + rv) + ring * 2 * rt) + 2 * a.B * a.Hq * a.D * 4
+
+
+def sweep(a, c, kv, kf, vf, tf, W, dev, gen):
+    import torch
+    from quantized_mixed_precision_qx_b200 import kvq
+    q = torch.randn(a.B, a.Hq, a.D, device=dev, generator=gen) / math.sqrt(a.D)
+    out = torch.empty_like(q)
+    ws = c.ensure_workspace(1)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clean = torch.ones(64 << 20, dtype=torch.int32, device=dev) if a.clean_flush else None
+    chunks = [kv(a.step) for _ in range(a.n // a.step)]
+    res = {}
+    for rep in range(a.warmup + a.reps):
+        kvq.kvq_cache_bind(c.handle, c.dev, c.nbytes)
+        for i, (k, v) in enumerate(chunks):
+            c.append(0, k, v)
+            flush.fill_(rep & 0xFF)
+            if clean is not None:
+                clean.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kvq.kvq_decode_attention(c.handle, 0, q, 1.0, out, ws, ws.numel())
+            e1.record()
+            torch.cuda.synchronize()
+            if rep >= a.warmup:
+                res.setdefault(i, []).append(e0.elapsed_time(e1) / 1e3)
+    for i, ts in sorted(res.items()):
+        n = (i + 1) * a.step
+        tm = statistics.median(ts)
+        nb = decode_bytes(a, n, kf, vf, tf, W)
+        print(json.dumps({"op": "decode", "n": n, "us": tm * 1e6, "gbs": nb / tm / 1e9,
+                          "algorithmic_bytes": nb}), flush=True)
 
 
 if __name__ == "__main__":
