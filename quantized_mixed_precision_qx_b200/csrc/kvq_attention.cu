@@ -252,14 +252,17 @@ size_t partial_floats(int G, int D) { return (size_t)G * (D + 2); }
 
 bool use_tensor_cores(int D) { return D == 128 || D == 256; }
 
-SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, bool tc) {
+int tc_ctas_per_sm(int head_dim) { return tc::min_ctas(head_dim / 32); }
+
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int tc_ctas) {
     SplitPlan p{};
-    const long long target = (tc ? 3LL : 4LL) * num_sms;
+    const bool tc = tc_ctas > 0;
+    const long long target = (tc ? (long long)tc_ctas : 4LL) * num_sms;
     long long per_unit = (target + units - 1) / units;
     if (per_unit < 1) per_unit = 1;
     if (tc) {
         // every split of either region gets the same number of tiles, chosen so that both
-        // regions' splits fit in about one wave (per_unit per unit, 3 CTAs per SM): the ring
+        // regions' splits fit in about one wave (per_unit per unit, tc_ctas CTAs per SM): the ring
         // pass and the low-bit pass then run side by side and end together
         const long long tr = (n_ring + tc::TOK - 1) / tc::TOK, tm = (n_main + tc::TOK - 1) / tc::TOK;
         long long per = (tr + tm + per_unit - 1) / per_unit;
@@ -340,7 +343,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
             t.D = lv.D;
             t.dependent = launched ? 1 : 0;
             const dim3 grid(ns, lv.H, lv.B * rows);
-            e = tc::launch_tc(fk.id, fv.id, t, grid, tc::smem_bytes(fk.stride, fv.stride, lv.D), st);
+            e = tc::launch_tc(fk.id, fv.id, t, grid, tc::smem_bytes(fk.stride, fv.stride, lv.D, tc::query_parts(fk.id)), st);
         } else {
             switch (CPL) {
                 case 1: e = run_pass1<1>(a, ns, lv.B, st); break;

@@ -1,26 +1,32 @@
 // kvq_decode_tc.cuh -- split-K decode / row-batched prefill pass 1 on warp-level tensor
 // cores, for head_dim 128 or 256 (nb = 4 or 8 blocks of 32 channels).
 //
-// CTA = 4 consumer warps + 1 producer warp. The producer streams the split's rows in
-// 64-row tiles with 1-D bulk copies (TMA engine) into a 3-stage shared-memory ring
+// CTA = 8 consumer warps + 1 producer warp. The producer streams the split's rows in
+// 64-row tiles with 1-D bulk copies (TMA engine) into a 2-stage shared-memory ring
 // (K tile and V tile are each one contiguous copy, since a region stores its rows back
-// to back). Each consumer warp takes 16 rows of every tile:
-//   S^T[16 x 8] = K[16 x D] Q^T[D x 8]   (m16n8k16; rows = tokens, 8 = the G <= 8 heads)
-//   p = exp2(S - m) with a per-head running max m and sum l (online softmax)
-//   O^T[D x 8] += V^T[D x 16] P^T[16 x 8]
-// Codes enter the MMAs exactly (fp16 integers); block scales are applied to the QK
-// accumulators per 32-channel block and folded into P for PV; the query and P*d are
-// split into hi + lo fp16 parts. At the end the 4 warps' states are merged in shared
-// memory and the CTA writes one (m, l, o) partial per head, like the CUDA-core path.
+// to back). A tile has 4 groups of 16 rows; each group is shared by a pair of consumer
+// warps, one per half of the channel blocks:
+//   S^T[16 x 8] = K[16 x D] Q^T[D x 8]   (m16n8k16; rows = tokens, 8 = the G <= 8 heads),
+//       each warp of the pair summing its half of the blocks; the two halves are
+//       exchanged through shared memory, so both warps hold the same S
+//   p = exp2(S - m) with a per-head running max m and sum l (online softmax; computed
+//       identically by both warps of the pair)
+//   O^T[D/2 x 8] += V^T[D/2 x 16] P^T[16 x 8]   (each warp: the output channels of its half)
+// Codes enter the MMAs exactly (fp16 integers); K block scales are applied to the QK
+// accumulators per 32-channel block, V block scales are folded into the V operand as an
+// exact hi + lo fp16 pair; the query and P are split into hi + lo parts. At the end the
+// 4 row groups' states are merged in shared memory and the CTA writes one (m, l, o)
+// partial per head, like the CUDA-core path.
 #pragma once
 #include "kvq_mma.cuh"
 
 namespace kvq {
 namespace tc {
 
-constexpr int TOK = 64;         // rows per stage
+constexpr int TOK = 64;                  // rows per stage
 constexpr int STAGES = 2;
-constexpr int CWARPS = 4;       // consumer warps
+constexpr int TGROUPS = TOK / 16;        // 16-row groups of a tile
+constexpr int CWARPS = 2 * TGROUPS;      // consumer warps: (row group, channel half)
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr int NBMAX = 8;
 // Lazy rescale: a head's running max is only raised when a score exceeds it by more
@@ -54,29 +60,48 @@ struct Args {
 };
 
 __host__ __device__ constexpr size_t stage_bytes(int ks, int vs) { return (size_t)TOK * (ks + vs); }
-// shared memory: [stages | final combine (aliased)] [P transpose] [mbarriers] [fault word]
+// shared memory: [stages | final combine (aliased)] [P transpose] [S exchange]
+//                [query fragments] [query sums] [mbarriers] [fault word]
 __host__ __device__ constexpr size_t comb_bytes(int D) {
-    return (size_t)(CWARPS * 8 * 3 + 16 + CWARPS * 8 * NBMAX + CWARPS * 8 * D) * sizeof(float);
+    return (size_t)(TGROUPS * 8 * 3 + 16 + TGROUPS * 8 * NBMAX + TGROUPS * 8 * D) * sizeof(float);
 }
 __host__ __device__ constexpr size_t main_bytes(int ks, int vs, int D) {
     return ((STAGES * stage_bytes(ks, vs) > comb_bytes(D) ? STAGES * stage_bytes(ks, vs) : comb_bytes(D)) + 127) & ~(size_t)127;
 }
 constexpr size_t PT_BYTES = CWARPS * 16 * 8 * sizeof(float);
-constexpr size_t QS_BYTES = NBMAX * 2 * 3 * 32 * sizeof(uint2);     // query fragments (<= 3 parts)
+constexpr size_t XS_BYTES = 2 * CWARPS * 32 * sizeof(float4);       // double-buffered S halves
+__host__ __device__ constexpr int query_parts(int kf) { return kf == F_BF16 ? 3 : 2; }
+__host__ __device__ constexpr size_t qs_bytes(int parts) { return (size_t)NBMAX * 2 * parts * 32 * sizeof(uint2); }
 constexpr size_t QSUM_BYTES = NBMAX * 8 * sizeof(float);
-__host__ __device__ constexpr size_t smem_bytes(int ks, int vs, int D) {
-    return main_bytes(ks, vs, D) + PT_BYTES + QS_BYTES + QSUM_BYTES + 2 * STAGES * sizeof(uint64_t) + 16;
+__host__ __device__ constexpr size_t smem_bytes(int ks, int vs, int D, int parts) {
+    return main_bytes(ks, vs, D) + PT_BYTES + XS_BYTES + qs_bytes(parts) + QSUM_BYTES + 2 * STAGES * sizeof(uint64_t) + 16;
 }
 
+// OR of `pred` over the 64 threads of a warp pair (named barrier `id`); also orders the
+// pair's shared-memory accesses like bar.sync
+__device__ __forceinline__ bool pair_any(int id, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 64, p;\n selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id) : "memory");
+    return r != 0;
+}
+
+// CTAs per SM the register allocation is sized for: head_dim 256 keeps 2 (no spills),
+// head_dim 128 fits 3
+__host__ __device__ constexpr int min_ctas(int nb) { return nb == 8 ? 2 : 3; }
+
 template <int KF, int VF, int NB>
-__global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
+__global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     using namespace mma;
     using KT = Fmt<KF>;
     using VT = Fmt<VF>;
     static_assert(KT::is_bf16 == VT::is_bf16, "K and V must use the same MMA operand type");
+    static_assert(NB % 2 == 0 && NB <= CWARPS, "two channel halves; one query block per warp");
     constexpr int KP = KT::parts;            // parts of the query split
     constexpr int VP = VT::parts;            // parts of the P split
     constexpr bool VSCALED = !VT::is_float;  // block scale folded into the V operand
+    constexpr int HB = NB / 2;               // blocks per channel half
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int D = 32 * NB, G = a.G, H = a.H;
@@ -84,14 +109,16 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     const size_t mb = main_bytes(a.kstride, a.vstride, D);
     uint8_t* stage0 = smem;
     float* pT = reinterpret_cast<float*>(smem + mb);                                   // [CWARPS][16][8]
-    uint2* qs = reinterpret_cast<uint2*>(smem + mb + PT_BYTES);                        // [NB][2][KP][32]
-    float* qsum_s = reinterpret_cast<float*>(smem + mb + PT_BYTES + QS_BYTES);         // [NB][8]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + QS_BYTES + QSUM_BYTES);
+    float4* xs = reinterpret_cast<float4*>(smem + mb + PT_BYTES);                      // [2][CWARPS][32]
+    uint2* qs = reinterpret_cast<uint2*>(smem + mb + PT_BYTES + XS_BYTES);             // [NB][2][KP][32]
+    float* qsum_s = reinterpret_cast<float*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP));   // [NB][8]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP) + QSUM_BYTES);
     uint64_t* empty = full + STAGES;
     int* fault = reinterpret_cast<int*>(empty + STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int tg = warp % TGROUPS, hf = warp / TGROUPS;     // consumer: row group, channel half
     const int h = blockIdx.y, br = blockIdx.z;
     const int b = br / a.rows, r = br % a.rows;
     const int split = blockIdx.x;
@@ -111,22 +138,15 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // query values of this lane's fragments, loaded first so their latency overlaps the setup
-    constexpr int QB = (NB + CWARPS - 1) / CWARPS;
-    float qv[QB][2][4];
-    if (warp < CWARPS) {
+    // query values of this lane's fragments (warp w builds block w), loaded first so their
+    // latency overlaps the setup
+    float qv[2][4];
+    if (warp < NB) {
         const float* qg = a.q + ((long long)br * G * H + (long long)h * G + g) * D;
 #pragma unroll
-        for (int bi = 0; bi < QB; ++bi) {
-            const int bb = warp + CWARPS * bi;
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
-#pragma unroll
-                for (int sl = 0; sl < 4; ++sl) {
-                    const int c = 32 * bb + q_channel<KF>(t, m, sl);
-                    qv[bi][m][sl] = (bb < NB && g < G) ? qg[c] : 0.f;
-                }
-        }
+            for (int sl = 0; sl < 4; ++sl) qv[m][sl] = (g < G) ? qg[32 * warp + q_channel<KF>(t, m, sl)] : 0.f;
     }
     // Rows past the end of a partial last tile are read (and multiplied by p = 0): zero
     // them in that tile's stage so they always hold finite values.
@@ -168,29 +188,23 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     }
 
     // ------------------------------------------------------------ query fragments
-    // (B operand of QK, head g of lane (g, t)), built while the first tiles are in flight:
-    // consumer warp w builds blocks w, w + 4 (and the asymmetric-format query sums),
-    // then the consumer warps meet at a named barrier.
+    // (B operand of QK, head g of lane (g, t)), built while the first tiles are in flight
     if (warp < CWARPS) {
+        if (warp < NB) {
 #pragma unroll
-        for (int bi = 0; bi < QB; ++bi) {
-            const int bb = warp + CWARPS * bi;
-            if (bb < NB) {
+            for (int m = 0; m < 2; ++m) {
+                float v[4];
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    float v[4];
-#pragma unroll
-                    for (int sl = 0; sl < 4; ++sl) {
-                        float x = qv[bi][m][sl] * a.qscale;
-                        if (kvarn) x *= sK[32 * bb + q_channel<KF>(t, m, sl)];
-                        v[sl] = x;
-                    }
-                    uint32_t p01[3], p23[3];
-                    split_pack<KF>(v[0], v[1], p01);
-                    split_pack<KF>(v[2], v[3], p23);
-#pragma unroll
-                    for (int pp = 0; pp < KP; ++pp) qs[((bb * 2 + m) * KP + pp) * 32 + lane] = make_uint2(p01[pp], p23[pp]);
+                for (int sl = 0; sl < 4; ++sl) {
+                    float x = qv[m][sl] * a.qscale;
+                    if (kvarn) x *= sK[32 * warp + q_channel<KF>(t, m, sl)];
+                    v[sl] = x;
                 }
+                uint32_t p01[3], p23[3];
+                split_pack<KF>(v[0], v[1], p01);
+                split_pack<KF>(v[2], v[3], p23);
+#pragma unroll
+                for (int pp = 0; pp < KP; ++pp) qs[((warp * 2 + m) * KP + pp) * 32 + lane] = make_uint2(p01[pp], p23[pp]);
             }
         }
         if constexpr (KT::asym) {
@@ -213,76 +227,90 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     }
 
     // ------------------------------------------------------------ consumers
-    float o[NB][2][4];
+    float o[HB][2][4];
     float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
-    float pm[NB];                         // asym V: sum_t p_t m_t,b for head g
+    float pm[HB];                         // asym V: sum_t p_t m_t,b for head g
 #pragma unroll
-    for (int bb = 0; bb < NB; ++bb) {
-        pm[bb] = 0.f;
+    for (int j = 0; j < HB; ++j) {
+        pm[j] = 0.f;
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o[bb][m][i] = 0.f;
+            for (int i = 0; i < 4; ++i) o[j][m][i] = 0.f;
     }
 
     if (warp < CWARPS) {
         float* myT = pT + warp * 128;
+        const int b0 = hf * HB;                      // first block of this warp's half
+        const int pair_bar = 2 + tg;                 // named barrier of the row-group pair
+        // ring slot s holds position n - W + ((s + W - n mod W) mod W)
         const long long W = a.W;
-        const long long ring_base = a.n - W;
+        const long long nmodw = a.ring ? a.n % W : 0;
+        const int sub0 = 16 * tg;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % STAGES;
-            if (!mbar_wait(&full[s], (it / STAGES) & 1)) { *fault = 1; break; }
+            const bool ok = mbar_wait(&full[s], (it / STAGES) & 1);
             const long long r0 = t0 + (long long)it * TOK;
             const int nrows = (int)min((long long)TOK, t1 - r0);
-            const int sub0 = 16 * warp;
-            if (sub0 < nrows) {
+            if (sub0 < nrows) {                      // uniform over the pair
                 const uint8_t* kt = stage0 + s * sb;
                 const uint8_t* vt = kt + (size_t)TOK * a.kstride;
                 auto valid = [&](int rr) -> bool {
                     if (sub0 + rr >= nrows) return false;
                     if (a.ring) {
-                        const long long slot = r0 + sub0 + rr;
-                        const long long pos = ring_base + ((slot - ring_base) % W + W) % W;
-                        return pos <= limit;
+                        long long d = r0 + sub0 + rr + W - nmodw;
+                        if (d >= W) d -= W;
+                        return a.n - W + d <= limit;
                     }
                     return true;
                 };
-                // ---------------- S^T = K Q^T
+                // ---------------- S^T = K Q^T over this warp's blocks
                 const uint8_t* rg = kt + (size_t)(sub0 + g) * a.kstride;
                 const uint8_t* rg8 = kt + (size_t)(sub0 + g + 8) * a.kstride;
                 float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (ok) {
 #pragma unroll
-                for (int bb = 0; bb < NB; ++bb) {
-                    uint32_t af[2][4];
-                    k_frags<KF>(rg, rg8, NB, bb, t, af);
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int j = 0; j < HB; ++j) {
+                        const int bb = b0 + j;
+                        uint32_t af[2][4];
+                        k_frags<KF>(rg, rg8, NB, bb, t, af);
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < 2; ++m)
+                        for (int m = 0; m < 2; ++m)
 #pragma unroll
-                        for (int pp = 0; pp < KP; ++pp) {
-                            const uint2 qv = qs[((bb * 2 + m) * KP + pp) * 32 + lane];
-                            mma_f<KF>(acc, af[m], qv.x, qv.y);
-                        }
-                    if constexpr (KT::is_float) {
+                            for (int pp = 0; pp < KP; ++pp) {
+                                const uint2 qv2 = qs[((bb * 2 + m) * KP + pp) * 32 + lane];
+                                mma_f<KF>(acc, af[m], qv2.x, qv2.y);
+                            }
+                        if constexpr (KT::is_float) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) sc[i] += acc[i];
-                    } else {
-                        const float dg = h2f_lo(reinterpret_cast<const uint16_t*>(rg)[bb]);
-                        const float dg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8)[bb]);
-                        sc[0] = fmaf(acc[0], dg, sc[0]);
-                        sc[1] = fmaf(acc[1], dg, sc[1]);
-                        sc[2] = fmaf(acc[2], dg8, sc[2]);
-                        sc[3] = fmaf(acc[3], dg8, sc[3]);
-                        if constexpr (KT::asym) {
-                            const float mg = h2f_lo(reinterpret_cast<const uint16_t*>(rg + KT::off_m(NB))[bb]);
-                            const float mg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8 + KT::off_m(NB))[bb]);
-                            const float2 qq = *reinterpret_cast<const float2*>(&qsum_s[bb * 8 + 2 * t]);
-                            sc[0] = fmaf(mg, qq.x, sc[0]);
-                            sc[1] = fmaf(mg, qq.y, sc[1]);
-                            sc[2] = fmaf(mg8, qq.x, sc[2]);
-                            sc[3] = fmaf(mg8, qq.y, sc[3]);
+                            for (int i = 0; i < 4; ++i) sc[i] += acc[i];
+                        } else {
+                            const float dg = h2f_lo(reinterpret_cast<const uint16_t*>(rg)[bb]);
+                            const float dg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8)[bb]);
+                            sc[0] = fmaf(acc[0], dg, sc[0]);
+                            sc[1] = fmaf(acc[1], dg, sc[1]);
+                            sc[2] = fmaf(acc[2], dg8, sc[2]);
+                            sc[3] = fmaf(acc[3], dg8, sc[3]);
+                            if constexpr (KT::asym) {
+                                const float mg = h2f_lo(reinterpret_cast<const uint16_t*>(rg + KT::off_m(NB))[bb]);
+                                const float mg8 = h2f_lo(reinterpret_cast<const uint16_t*>(rg8 + KT::off_m(NB))[bb]);
+                                const float2 qq = *reinterpret_cast<const float2*>(&qsum_s[bb * 8 + 2 * t]);
+                                sc[0] = fmaf(mg, qq.x, sc[0]);
+                                sc[1] = fmaf(mg, qq.y, sc[1]);
+                                sc[2] = fmaf(mg8, qq.x, sc[2]);
+                                sc[3] = fmaf(mg8, qq.y, sc[3]);
+                            }
                         }
                     }
+                }
+                // ---------------- exchange the halves (and any wait failure) within the pair
+                float4* xb = xs + (it & 1) * CWARPS * 32;
+                xb[warp * 32 + lane] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+                if (pair_any(pair_bar, !ok)) { *fault = 1; break; }
+                {
+                    const float4 ps = xb[(warp ^ TGROUPS) * 32 + lane];
+                    sc[0] += ps.x; sc[1] += ps.y; sc[2] += ps.z; sc[3] += ps.w;   // commutative: same in both
                 }
                 if (!valid(g)) { sc[0] = -INFINITY; sc[1] = -INFINITY; }
                 if (!valid(g + 8)) { sc[2] = -INFINITY; sc[3] = -INFINITY; }
@@ -303,11 +331,11 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
                     lrun[0] *= c0;
                     lrun[1] *= c1;
 #pragma unroll
-                    for (int bb = 0; bb < NB; ++bb)
+                    for (int j = 0; j < HB; ++j)
 #pragma unroll
                         for (int m = 0; m < 2; ++m) {
-                            o[bb][m][0] *= c0; o[bb][m][1] *= c1;
-                            o[bb][m][2] *= c0; o[bb][m][3] *= c1;
+                            o[j][m][0] *= c0; o[j][m][1] *= c1;
+                            o[j][m][2] *= c0; o[j][m][3] *= c1;
                         }
                     if constexpr (VT::asym) {
                         // pm belongs to head g: fetch that head's factor from lane (g >> 1)
@@ -315,7 +343,7 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
                         const float f1 = __shfl_sync(0xffffffffu, c1, g >> 1);
                         const float cg = (g & 1) ? f1 : f0;
 #pragma unroll
-                        for (int bb = 0; bb < NB; ++bb) pm[bb] *= cg;
+                        for (int j = 0; j < HB; ++j) pm[j] *= cg;
                     }
                     mrun[0] = mn0;
                     mrun[1] = mn1;
@@ -352,29 +380,30 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
 #pragma unroll
                     for (int pp = 0; pp < 3; ++pp) { bp[pp][0] = x01[pp]; bp[pp][1] = x23[pp]; }
                 }
-                // ---------------- O^T += V^T P^T
+                // ---------------- O^T += V^T P^T over this warp's blocks
 #pragma unroll
-                for (int bb = 0; bb < NB; ++bb) {
+                for (int j = 0; j < HB; ++j) {
+                    const int bb = b0 + j;
                     if constexpr (VSCALED) {
                         uint32_t ah[2][4], al[2][4];
                         v_frags_scaled<VF>(vr0, vr1, vr2, vr3, NB, bb, g, ah, al);
 #pragma unroll
                         for (int m = 0; m < 2; ++m) {
-                            mma_f16(o[bb][m], ah[m], bp[0][0], bp[0][1]);
-                            mma_f16(o[bb][m], ah[m], bp[1][0], bp[1][1]);
-                            mma_f16(o[bb][m], al[m], bp[0][0], bp[0][1]);
+                            mma_f16(o[j][m], ah[m], bp[0][0], bp[0][1]);
+                            mma_f16(o[j][m], ah[m], bp[1][0], bp[1][1]);
+                            mma_f16(o[j][m], al[m], bp[0][0], bp[0][1]);
                         }
                         if constexpr (VT::asym) {
                             const float m0 = h2f_lo(reinterpret_cast<const uint16_t*>(vr0 + VT::off_m(NB))[bb]);
                             const float m1 = h2f_lo(reinterpret_cast<const uint16_t*>(vr1 + VT::off_m(NB))[bb]);
                             const float m2 = h2f_lo(reinterpret_cast<const uint16_t*>(vr2 + VT::off_m(NB))[bb]);
                             const float m3 = h2f_lo(reinterpret_cast<const uint16_t*>(vr3 + VT::off_m(NB))[bb]);
-                            float acc = pm[bb];
+                            float acc = pm[j];
                             if (v0) acc = fmaf(pv[0], m0, acc);
                             if (v1) acc = fmaf(pv[1], m1, acc);
                             if (v2) acc = fmaf(pv[2], m2, acc);
                             if (v3) acc = fmaf(pv[3], m3, acc);
-                            pm[bb] = acc;
+                            pm[j] = acc;
                         }
                     } else {
                         uint32_t af[2][4];
@@ -382,70 +411,79 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
 #pragma unroll
                         for (int m = 0; m < 2; ++m)
 #pragma unroll
-                            for (int pp = 0; pp < VP; ++pp) mma_f<VF>(o[bb][m], af[m], bp[pp][0], bp[pp][1]);
+                            for (int pp = 0; pp < VP; ++pp) mma_f<VF>(o[j][m], af[m], bp[pp][0], bp[pp][1]);
                     }
                 }
+            } else if (!ok) {
+                *fault = 1;
+                break;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
 
-    // ------------------------------------------------------------ combine the 4 warps
+    // ------------------------------------------------------------ combine the 4 row groups
     __syncthreads();
-    // shared layout (reusing the stages): cm[CWARPS][8], cl[CWARPS][8], cpm[CWARPS][8][NBMAX], co[CWARPS][8][D]
+    // shared layout (reusing the stages): cm[TGROUPS][8], cl[TGROUPS][8],
+    // cpm[TGROUPS][8][NBMAX], co[TGROUPS][8][D]
     float* cm = reinterpret_cast<float*>(smem);
-    float* cl = cm + CWARPS * 8;
-    float* cpm = cl + CWARPS * 8;
-    float* co = cpm + CWARPS * 8 * NBMAX;
+    float* cl = cm + TGROUPS * 8;
+    float* cpm = cl + TGROUPS * 8;
+    float* co = cpm + TGROUPS * 8 * NBMAX;
     if (warp < CWARPS) {
-        // l: reduce the per-thread partial sums over the 8 lanes sharing t
-        float l0 = lrun[0], l1 = lrun[1];
+        const int b0 = hf * HB;
+        if (hf == 0) {
+            // l: reduce the per-thread partial sums over the 8 lanes sharing t (the pair
+            // holds identical m and l)
+            float l0 = lrun[0], l1 = lrun[1];
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-        }
-        if (g == 0) {
-            cm[warp * 8 + 2 * t] = mrun[0];
-            cm[warp * 8 + 2 * t + 1] = mrun[1];
-            cl[warp * 8 + 2 * t] = l0;
-            cl[warp * 8 + 2 * t + 1] = l1;
+            for (int off = 4; off < 32; off <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+            }
+            if (g == 0) {
+                cm[tg * 8 + 2 * t] = mrun[0];
+                cm[tg * 8 + 2 * t + 1] = mrun[1];
+                cl[tg * 8 + 2 * t] = l0;
+                cl[tg * 8 + 2 * t + 1] = l1;
+            }
         }
         if constexpr (VT::asym) {
 #pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-                float v = pm[bb];
+            for (int j = 0; j < HB; ++j) {
+                float v = pm[j];
                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                 v += __shfl_xor_sync(0xffffffffu, v, 2);
-                if (t == 0) cpm[(warp * 8 + g) * NBMAX + bb] = v;
+                if (t == 0) cpm[(tg * 8 + g) * NBMAX + b0 + j] = v;
             }
         }
 #pragma unroll
-        for (int bb = 0; bb < NB; ++bb) {
+        for (int j = 0; j < HB; ++j) {
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
-                const int c_lo = 32 * bb + v_channel(g, m, 0), c_hi = 32 * bb + v_channel(g, m, 1);
-                co[(warp * 8 + 2 * t) * D + c_lo] = o[bb][m][0];
-                co[(warp * 8 + 2 * t + 1) * D + c_lo] = o[bb][m][1];
-                co[(warp * 8 + 2 * t) * D + c_hi] = o[bb][m][2];
-                co[(warp * 8 + 2 * t + 1) * D + c_hi] = o[bb][m][3];
+                const int c_lo = 32 * (b0 + j) + v_channel(g, m, 0), c_hi = 32 * (b0 + j) + v_channel(g, m, 1);
+                co[(tg * 8 + 2 * t) * D + c_lo] = o[j][m][0];
+                co[(tg * 8 + 2 * t + 1) * D + c_lo] = o[j][m][1];
+                co[(tg * 8 + 2 * t) * D + c_hi] = o[j][m][2];
+                co[(tg * 8 + 2 * t + 1) * D + c_hi] = o[j][m][3];
             }
         }
     }
-    // per head: max over the warps, each warp's weight and the weighted sum of l
-    float* cw = co + CWARPS * 8 * D;      // [CWARPS][8]
-    float* cM = cw + CWARPS * 8;          // [8]
+    __syncthreads();
+    // per head: max over the row groups, each group's weight and the weighted sum of l
+    float* cw = co + TGROUPS * 8 * D;     // [TGROUPS][8]
+    float* cM = cw + TGROUPS * 8;         // [8]
     float* cL = cM + 8;                   // [8]
     const bool bad = *fault != 0;
     if (threadIdx.x < 8) {
         const int hh = threadIdx.x;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, cm[w * 8 + hh]);
+        for (int w = 0; w < TGROUPS; ++w) M = fmaxf(M, cm[w * 8 + hh]);
         float L = 0.f;
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) {
+        for (int w = 0; w < TGROUPS; ++w) {
             const float mw = cm[w * 8 + hh];
             const float e = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2(mw - M);
             cw[w * 8 + hh] = e;
@@ -456,12 +494,12 @@ __global__ void __launch_bounds__(THREADS, 3) decode_tc(Args a) {
     }
     __syncthreads();
     float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
-    // o = sum over warps of weight * o_w, two channels per thread step (8-byte stores)
+    // o = sum over row groups of weight * o_w, two channels per thread step (8-byte stores)
     for (int idx = 2 * threadIdx.x; idx < G * D; idx += 2 * THREADS) {
         const int hh = idx / D, c = idx % D;
         float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) {
+        for (int w = 0; w < TGROUPS; ++w) {
             const float e = cw[w * 8 + hh];
             float2 ow = *reinterpret_cast<const float2*>(&co[(w * 8 + hh) * D + c]);
             if constexpr (VT::asym) {

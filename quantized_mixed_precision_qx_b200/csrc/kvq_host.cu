@@ -233,7 +233,8 @@ static kvq_status attention_common(kvq_cache* c, int32_t layer, const float* q, 
     const LayerView lv = layer_view(c, layer);
     const long long n_ring = c->W ? (n < c->W ? n : c->W) : 0;
     const long long units = (long long)c->L.batch * c->L.n_kv_heads * rows;
-    const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, use_tensor_cores(c->L.head_dim));
+    const int tc_ctas = use_tensor_cores(c->L.head_dim) ? tc_ctas_per_sm(c->L.head_dim) : 0;
+    const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, tc_ctas);
     return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, rows, plan, (cudaStream_t)stream));
 }
 

@@ -102,7 +102,9 @@ struct SplitPlan {
     int n_split() const { return n_main_split + n_ring_split; }
 };
 // Tensor-core path (head_dim 128 / 256) when tc is set: splits are whole 64-row tiles.
-SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, bool tc);
+// tc_ctas: CTAs per SM of the tensor-core decode kernel (0: CUDA-core path)
+SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int num_sms, int tc_ctas);
+int tc_ctas_per_sm(int head_dim);
 bool use_tensor_cores(int D);
 size_t partial_floats(int G, int D);   // floats of one split partial
 
