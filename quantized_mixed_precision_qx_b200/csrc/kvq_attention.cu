@@ -258,7 +258,8 @@ SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int n
     SplitPlan p{};
     const bool tc = tc_ctas > 0;
     const long long target = (tc ? (long long)tc_ctas : 4LL) * num_sms;
-    long long per_unit = (target + units - 1) / units;
+    // rounded down: units * per_unit CTAs must not spill into a second wave
+    long long per_unit = target / units;
     if (per_unit < 1) per_unit = 1;
     if (tc) {
         // every split of either region gets the same number of tiles, chosen so that both
@@ -267,6 +268,8 @@ SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int n
         const long long tr = (n_ring + tc::TOK - 1) / tc::TOK, tm = (n_main + tc::TOK - 1) / tc::TOK;
         long long per = (tr + tm + per_unit - 1) / per_unit;
         if (per < 1) per = 1;
+        // each region rounds its split count up: grow the tile count until both fit
+        while ((tr + per - 1) / per + (tm + per - 1) / per > per_unit && per < tr + tm) ++per;
         p.ring_chunk = p.main_chunk = per * tc::TOK;
         p.n_ring_split = (int)((tr + per - 1) / per);
         p.n_main_split = (int)((tm + per - 1) / per);
