@@ -167,8 +167,8 @@ attn_pass1(P1Args a) {
 }
 
 // Merge of the split partials. One CTA per (b, row, q head) and 32-channel slice; its
-// 256 threads are 32 channels x 8 split groups. Group j folds splits j, j+8, j+16, ... in
-// order with an online rescale (one pass over m, l and o), then the 8 groups are folded
+// 32 * MG threads are 32 channels x MG split groups. Group j folds splits j, j+MG, ... in
+// order with an online rescale (one pass over m, l and o), then the MG groups are folded
 // in a fixed order, so the result is bit-reproducible.
 constexpr int MG = 16;
 constexpr int MU = 4;   // partials per merge step
