@@ -207,6 +207,24 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------ ranks
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank times over all ranks (every rank gets the result).
+    The tensor lives on `device` (a CUDA device under NCCL, the CPU under gloo)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbs(world, bytes_per_rank, max_seconds):
+    """Whole-job throughput of `world` replicas that each moved `bytes_per_rank` algorithmic
+    bytes, timed as the slowest rank (weak scaling)."""
+    return world * bytes_per_rank / max_seconds / 1e9
+
+
 # ------------------------------------------------------------------------ CUDA arm
 def run_kvq(args, rank, world):
     import torch
@@ -323,15 +341,12 @@ def run_kvq(args, rank, world):
     d2h = n_steps * B_ * HQ_ * D_ * 4
 
     # ---- max over ranks
-    t = torch.tensor([dec_t, app_t, e2e_s, step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    dec_t, app_t, e2e_s, step_ms = t.tolist()
+    dec_t, app_t, e2e_s, step_ms = max_over_ranks([dec_t, app_t, e2e_s, step_ms], world, dev)
 
     if rank != 0:
         return
     peak, peak_kind = read_peaks()
-    value = world * dec_bytes * args.steps / dec_t / 1e9
+    value = whole_job_gbs(world, dec_bytes * args.steps, dec_t)
     achieved = dec_bytes * args.steps / dec_t / 1e9          # per GPU
     traffic = recorded_traffic()
     extra = supplementary(dev, peak) if not args.no_extra else None
