@@ -6,18 +6,20 @@
 // with fp32 accumulators in tensor memory:
 //
 //   CTA   = 128 query rows of one (batch, kv head): row r = chunk row * G + head in group,
-//           TMEM lane r. 8 warps: warps 0-3 own one row per thread (softmax, epilogue);
-//           all 8 share the dequantization; its global loads run under the MMAs, with every load
-//           of a phase issued before its values are used.
-//   tile  = 64 key positions. Each tile is dequantized into shared memory as exact fp16
+//           TMEM lane r. 16 warps: warps 0-3 own one row per thread (softmax, epilogue);
+//           all share the dequantization.
+//   tile  = 32 key positions. Each tile is dequantized into shared memory as exact fp16
 //           hi + lo parts (K~ = hi + lo; the query and P are split the same way), and
-//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N64 K16 steps) -> TMEM cols [0, 64)
-//           O += Ph Vh + Ph Vl + Pl Vh    (3 passes, M128 N256 K16 steps) -> TMEM cols [256, 512)
+//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N32 K16 steps) -> TMEM cols [0, 32)
+//           O += Ph Vh + Ph Vl + Pl Vh    (3 passes, M128 N=D K16 steps) -> TMEM cols [256, 256 + D)
 //   The softmax is row-local (each thread owns its row), with a lazily raised running max.
+//   K~ and V~^T have buffers of their own, so the P V~ MMAs of a tile run while the next
+//   tile's K~ is dequantized and its S computed; the raw rows of tile i + 1 are fetched by
+//   bulk copies into the second staging buffer while tile i is processed.
 //
-// Shared memory (head_dim D = 32 NB): Q hi/lo 2 x 128 x D x 2 B, a K/V tile buffer
-// 2 x 64 x D x 2 B (K~ first, then V~^T), P hi/lo 2 x 128 x 64 x 2 B. All operands use the
-// K-major 128-byte-swizzled layout of kvq_tc5.cuh.
+// Shared memory (head_dim D = 32 NB): Q hi 128 x D x 2 B (Q lo lives in TMEM), 2 staging
+// buffers of 2 x 32 raw rows, K~ hi/lo 2 x 32 x D x 2 B (K-major, 128-byte swizzle),
+// V~^T hi/lo 2 x D x 32 x 2 B and P hi/lo 2 x 128 x 32 x 2 B (K-major, 64-byte swizzle).
 #include "kvq_internal.cuh"
 #include "kvq_mma.cuh"
 #include "kvq_tc5.cuh"
@@ -26,8 +28,8 @@ namespace kvq {
 namespace {
 
 constexpr int PM = 128;           // query rows per CTA
-constexpr int PN = 64;            // key positions per tile
-constexpr int PTHREADS = 256;     // 8 warps: warps 0-3 own the 128 TMEM rows, all dequantize
+constexpr int PN = 32;            // key positions per tile
+constexpr int PTHREADS = 512;     // 16 warps: 4 own the 128 TMEM rows, 11 dequantize, 1 issues
 constexpr float PF_RESCALE = 8.0f;
 
 struct PrefillArgs {
@@ -40,9 +42,12 @@ struct PrefillArgs {
     int* fault;                   // optional device fault word (may be null)
 };
 
+// raw rows of one tile (K half then V half of a staging buffer): the widest row is 2 D bytes
+__host__ __device__ constexpr size_t stage_half(int D) { return (size_t)PN * 2 * D; }
 __host__ __device__ constexpr size_t pf_smem(int D) {
-    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 65536 /* staging */ +
-           2 * (size_t)PN * D * 2 + 2 * (size_t)PM * PN * 2 + 64;
+    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 4 * stage_half(D) /* 2 staging buffers */ +
+           2 * (size_t)PN * D * 2 /* K~ */ + 2 * (size_t)D * PN * 2 /* V~^T */ + 2 * (size_t)PM * PN * 2 /* P */ + 128 /* barriers */ +
+           1024 /* tail pad: no operand read can pass the end of the allocation */;
 }
 
 // split fp32 -> fp16 hi (truncated to 11 significant bits) + fp16 lo (rounded remainder)
@@ -59,6 +64,16 @@ __device__ __forceinline__ void store_chunk(uint8_t* hi_tile, uint8_t* lo_tile, 
 #pragma unroll
     for (int j = 0; j < 8; ++j) split16(x[j], h[j], l[j]);
     const uint32_t off = t5::sw128_offset(row, k0, rows);
+    *reinterpret_cast<uint4*>(hi_tile + off) = *reinterpret_cast<const uint4*>(h);
+    *reinterpret_cast<uint4*>(lo_tile + off) = *reinterpret_cast<const uint4*>(l);
+}
+
+// same for a K-major tile with 64-byte rows (K extent 32)
+__device__ __forceinline__ void store_chunk64(uint8_t* hi_tile, uint8_t* lo_tile, int row, int k0, const float (&x)[8]) {
+    __align__(16) __half h[8], l[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) split16(x[j], h[j], l[j]);
+    const uint32_t off = t5::sw64_offset(row, k0);
     *reinterpret_cast<uint4*>(hi_tile + off) = *reinterpret_cast<const uint4*>(h);
     *reinterpret_cast<uint4*>(lo_tile + off) = *reinterpret_cast<const uint4*>(l);
 }
@@ -226,41 +241,54 @@ __device__ __forceinline__ void kperm8(const float (&x)[8], float (&y)[8]) {
     y[0] = x[0]; y[1] = x[4]; y[2] = x[1]; y[3] = x[5]; y[4] = x[2]; y[5] = x[6]; y[6] = x[3]; y[7] = x[7];
 }
 
-// Position order inside a 64-position tile: K~ row r, S / P column r and V~^T k-slot r all hold
-// position t0 + slot_pos(r), the 8 x 8 transpose of the natural order. A thread that fills k-slots
-// 8m .. 8m+7 of V~^T then reads staged rows m, m+8, .., m+56, so the 8 lanes with consecutive m
-// read consecutive rows (row strides are 16-byte multiples, so rows 8 apart share banks).
-__host__ __device__ constexpr int slot_pos(int r) { return ((r & 7) << 3) | (r >> 3); }
-static_assert(PN == 64, "slot_pos is the 8 x 8 transpose of a 64-position tile");
+// Position order inside a tile: K~ row r, S / P column r and V~^T k-slot r all hold
+// position t0 + slot_pos(r), the (PN/8) x 8 transpose of the natural order. A thread that
+// fills k-slots 8m .. 8m+7 of V~^T then reads staged rows m, m + PN/8, .., so lanes with
+// consecutive m read consecutive rows (row strides are 16-byte multiples, so rows PN/8
+// apart can share a shared-memory bank).
+__host__ __device__ constexpr int slot_pos(int r) { return ((r & 7) * (PN / 8)) | (r >> 3); }
+static_assert(PN % 8 == 0 && PN / 8 <= 8, "slot_pos needs 8-position groups");
 
-// Staging of one tile's raw rows (K rows then V rows), filled by bulk copies: positions
-// below the window come from the low-bit store, the others from the ring (in position
-// order, the ring slot range split at its wrap).
-struct Stage {
-    int t0, t_last;               // positions held
-    int n_main;                   // rows from the low-bit store (positions t0 .. t0 + n_main - 1)
-};
-constexpr int STAGE_HALF = 32 * 1024;   // K rows at [0, 32 KB), V rows at [32 KB, 64 KB)
+constexpr int OWNER_WARPS = 4;                       // softmax / epilogue: one query row per thread
+constexpr int DQ_WARPS = 11;                         // dequantization
+constexpr int ISSUER_WARP = OWNER_WARPS + DQ_WARPS;  // lane 0 issues the MMAs and the bulk copies
+static_assert(PTHREADS == 32 * (ISSUER_WARP + 1), "warp roles");
+
+// bounded wait whose outcome is the same for every lane of the warp
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mma::mbar_wait(bar, parity)) != 0;
+}
 
 template <int NB>
 __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     constexpr int D = 32 * NB;
     constexpr int CHUNKS = D / 8;                    // 8-channel chunks per row
+    constexpr size_t SH = stage_half(D);
     const LayerView& lv = a.lv;
     extern __shared__ uint8_t raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* q_hi = sm;                              // Q hi [PM x D]; Q lo lives in TMEM
-    uint8_t* stage = q_hi + PM * D * 2;              // raw rows of the next tile (64 KB)
-    uint8_t* kv_hi = stage + 2 * STAGE_HALF;         // K~ [PN x D], later V~^T [D x PN]
-    uint8_t* kv_lo = kv_hi + PN * D * 2;
-    uint8_t* p_hi = kv_lo + PN * D * 2;              // P [PM x PN]
+    uint8_t* stage = q_hi + PM * D * 2;              // 2 buffers x (K rows, V rows)
+    uint8_t* k_hi = stage + 4 * SH;                  // K~ [PN x D], 128-byte swizzle
+    uint8_t* k_lo = k_hi + PN * D * 2;
+    uint8_t* v_hi = k_lo + PN * D * 2;               // V~^T [D x PN], 64-byte swizzle
+    uint8_t* v_lo = v_hi + D * PN * 2;
+    uint8_t* p_hi = v_lo + D * PN * 2;               // P [PM x PN], 64-byte swizzle
     uint8_t* p_lo = p_hi + PM * PN * 2;
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);   // MMA completion
-    uint64_t* sbar = mbar + 1;                                          // staging copies
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbar + 1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);
+    uint64_t* st_full = bars;                        // [2] raw rows of a tile staged
+    uint64_t* s_full = bars + 2;                     // [2] S of a tile in TMEM buffer t % 2
+    uint64_t* s_empty = bars + 4;                    // [2] owners have read that S buffer
+    uint64_t* k_full = bars + 6;                     // K~ written
+    uint64_t* k_empty = bars + 7;                    // S MMAs done reading K~
+    uint64_t* v_full = bars + 8;                     // V~^T written (and the staging buffer consumed)
+    uint64_t* p_full = bars + 9;                     // P written
+    uint64_t* o_done = bars + 10;                    // P V~ MMAs done
+    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 11);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const bool owner = tid < PM;                     // owns TMEM lane / query row tid
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool owner = warp < OWNER_WARPS;           // owns TMEM lane / query row tid
     const int G = lv.G, H = lv.H;
     const int h = blockIdx.y, b = blockIdx.z;
     const int rows_total = a.C * G;
@@ -282,8 +310,17 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     const int n_tiles = tile_limit / PN + 1;
 
     if (tid == 0) {
-        mma::mbar_init(mbar, 1);
-        mma::mbar_init(sbar, 1);
+        for (int i = 0; i < 2; ++i) {
+            mma::mbar_init(&st_full[i], 1);
+            mma::mbar_init(&s_full[i], 1);
+            mma::mbar_init(&s_empty[i], OWNER_WARPS);
+        }
+        mma::mbar_init(k_full, DQ_WARPS);
+        mma::mbar_init(k_empty, 1);
+        mma::mbar_init(v_full, DQ_WARPS);
+        mma::mbar_init(p_full, OWNER_WARPS);
+        mma::mbar_init(o_done, 1);
+        *fault_flag = 0;
         mma::fence_mbar_init();
     }
     if (warp == 0) { t5::tmem_alloc(tmem_slot, 512); t5::tmem_relinquish(); }
@@ -291,48 +328,53 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem;                       // S: columns [0, 64)
+    const uint32_t t_s = tmem;                       // S: columns [0, PN) and [PN, 2 PN)
     const uint32_t t_qlo = tmem + 64;                // Q lo: columns [64, 64 + D/2)
     const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
 
-    // issue the bulk copies of tile `tile`'s raw rows into the staging buffer (thread 0)
+    // bulk copies of tile `tile`'s raw rows into staging buffer tile % 2 (issuer lane)
+    int st_last[2] = {-1, -1};                       // last tile staged per buffer
     auto issue_stage = [&](int tile) {
         const int t0 = tile * PN;
         const int tl = min(t0 + PN - 1, tile_limit);
         const int nm = max(0, min(tl + 1, ring0) - t0);       // rows from the low-bit store
         const int nr = (tl + 1 - t0) - nm;                    // rows from the ring
+        uint64_t* bar = &st_full[tile & 1];
         uint32_t bytes = 0;
+#pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
-            const SideView& v = kv ? vside : kside;
-            uint8_t* dst = stage + kv * STAGE_HALF;
-            if (nm > 0) {
-                const uint32_t cb = (uint32_t)nm * v.fmain.stride;
-                bytes += cb;
-            }
-            if (nr > 0) bytes += (uint32_t)nr * v.ftail.stride;
-            (void)dst;
+            const RowFmt fm = kv ? vside.fmain : kside.fmain;
+            const RowFmt ft = kv ? vside.ftail : kside.ftail;
+            if (nm > 0) bytes += (uint32_t)nm * fm.stride;
+            if (nr > 0) bytes += (uint32_t)nr * ft.stride;
         }
-        mma::mbar_arrive_expect_tx(sbar, bytes);
+        mma::mbar_arrive_expect_tx(bar, bytes);
+        if (tile & 1) st_last[1] = tile; else st_last[0] = tile;
+#pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
-            const SideView& v = kv ? vside : kside;
-            uint8_t* dst = stage + kv * STAGE_HALF;
+            const SideView v = kv ? vside : kside;
+            uint8_t* dst = stage + (size_t)(tile & 1) * 2 * SH + kv * SH;
             if (nm > 0) {
                 const uint32_t cb = (uint32_t)nm * v.fmain.stride;
-                mma::bulk_g2s(dst, v.main + (long long)t0 * v.fmain.stride, cb, sbar);
+                mma::bulk_g2s(dst, v.main + (long long)t0 * v.fmain.stride, cb, bar);
                 dst += cb;
             }
             if (nr > 0) {
                 const int p = t0 + nm;                         // first ring position
                 const int s0 = p % W;
                 const int c1 = min(nr, W - s0);
-                mma::bulk_g2s(dst, v.ring + (long long)s0 * v.ftail.stride, (uint32_t)c1 * v.ftail.stride, sbar);
+                mma::bulk_g2s(dst, v.ring + (long long)s0 * v.ftail.stride, (uint32_t)c1 * v.ftail.stride, bar);
                 if (nr > c1)
-                    mma::bulk_g2s(dst + (size_t)c1 * v.ftail.stride, v.ring, (uint32_t)(nr - c1) * v.ftail.stride, sbar);
+                    mma::bulk_g2s(dst + (size_t)c1 * v.ftail.stride, v.ring, (uint32_t)(nr - c1) * v.ftail.stride, bar);
             }
         }
     };
-    if (tid == 0) issue_stage(0);
+    const bool issuer = warp == ISSUER_WARP && lane == 0;
+    if (issuer) {
+        issue_stage(0);
+        if (n_tiles > 1) issue_stage(1);
+    }
 
     // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row)
     if (owner) {
@@ -365,13 +407,11 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             }
             t5::tmem_st32(t_qlo + lane_off + c64 / 2, cols);
         }
+        t5::fence_proxy_async();
     }
-
-    const uint32_t idesc_s = t5::idesc_f16(PM, PN);
-    const uint32_t idesc_o = t5::idesc_f16(PM, D);
-    const uint32_t sq_hi = t5::smem_addr(q_hi);
-    const uint32_t skv_hi = t5::smem_addr(kv_hi), skv_lo = t5::smem_addr(kv_lo);
-    const uint32_t sp_hi = t5::smem_addr(p_hi), sp_lo = t5::smem_addr(p_lo);
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
 
     // Tile modes (uniform over the CTA): 1 = every position in the low-bit store and its
     // format has a fast path, 2 = every position in the ring with a fast tail format,
@@ -384,187 +424,40 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     };
     // staged row of position t (clamped to the tile's last position)
     auto srow = [&](int kv, int t0, int t, uint32_t& sel) -> const uint8_t* {
-        const SideView& v = kv ? vside : kside;
+        const RowFmt fm = kv ? vside.fmain : kside.fmain;
+        const RowFmt ft = kv ? vside.ftail : kside.ftail;
         const int tl = min(t0 + PN - 1, tile_limit);
         t = min(t, tl);
         const int nm = max(0, min(tl + 1, ring0) - t0);
-        const uint8_t* base = stage + kv * STAGE_HALF;
-        if (t - t0 < nm) { sel = 0; return base + (size_t)(t - t0) * v.fmain.stride; }
+        const uint8_t* base = stage + (size_t)((t0 / PN) & 1) * 2 * SH + kv * SH;
+        if (t - t0 < nm) { sel = 0; return base + (size_t)(t - t0) * fm.stride; }
         sel = 1;
-        return base + (size_t)nm * v.fmain.stride + (size_t)(t - t0 - nm) * v.ftail.stride;
+        return base + (size_t)nm * fm.stride + (size_t)(t - t0 - nm) * ft.stride;
     };
+    auto set_fault = [&]() { *fault_flag = 1; };
 
     float m_run = -INFINITY, l_run = 0.f;
-    uint32_t phase = 0, sphase = 0;
-    bool have_o = false;
-    bool fault = false;
-    constexpr int PER = PN * CHUNKS / PTHREADS;      // K chunk units per thread
+    int s_last = -1, o_last = -1;                    // issuer: last tile whose S / P V~ MMAs were committed
 
-    t5::fence_before_sync();
-    __syncthreads();
-    t5::fence_after_sync();
-
-    for (int tile = 0; tile < n_tiles && !fault; ++tile) {
-        const int t0 = tile * PN;
-        // ---------------- wait for the staged raw rows of this tile
-        fault = __syncthreads_or((!mma::mbar_wait(sbar, sphase & 1)) || fault) != 0;
-        ++sphase;
-        if (fault) break;
-        // ---------------- K~ tile -> hi/lo (rows = positions, k = channels in chunk k order)
-        {
-            const int kmode = tile_mode(t0, kside);
-            const int fid = kmode == 1 ? kside.fmain.id : kside.ftail.id;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) {
-                const int u = tid + i * PTHREADS;
-                const int kr = u / CHUNKS, ch = u % CHUNKS;
-                uint32_t sel;
-                const uint8_t* row = srow(0, t0, t0 + slot_pos(kr), sel);
-                uint32_t out[8];
-                if (kmode != 0) {
-                    const int cb = ch >> 2, ct = ch & 3;
-                    switch (fid) {
-                        case F_Q2_0: k_chunk_fast<F_Q2_0, NB>(row, cb, ct, out); break;
-                        case F_Q3_0: k_chunk_fast<F_Q3_0, NB>(row, cb, ct, out); break;
-                        case F_Q4_0: k_chunk_fast<F_Q4_0, NB>(row, cb, ct, out); break;
-                        case F_Q5_0: k_chunk_fast<F_Q5_0, NB>(row, cb, ct, out); break;
-                        case F_Q6_0: k_chunk_fast<F_Q6_0, NB>(row, cb, ct, out); break;
-                        case F_Q8_0: k_chunk_fast<F_Q8_0, NB>(row, cb, ct, out); break;
-                        default: k_chunk_fast<F_F16, NB>(row, cb, ct, out); break;
-                    }
-                    const uint32_t off = t5::sw128_offset(kr, 8 * ch, PN);
-                    *reinterpret_cast<uint4*>(kv_hi + off) = make_uint4(out[0], out[1], out[2], out[3]);
-                    *reinterpret_cast<uint4*>(kv_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
-                } else {
-                    Raw8 rk;
-                    fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, rk);
-                    float x[8], y[8];
-                    decode_raw8(kside, rk, 8 * ch, x);
-                    kperm8(x, y);
-                    store_chunk(kv_hi, kv_lo, kr, 8 * ch, PN, y);
-                }
-            }
-        }
-        t5::fence_proxy_async();
-        t5::fence_before_sync();
-        __syncthreads();
-        t5::fence_after_sync();
-        // ---------------- S = Q K~^T: Qh Kh + Qh Kl (A from shared memory) + Ql Kh (A from TMEM)
-        if (tid == 0) {
-            int step = 0;
-#pragma unroll 1
-            for (int pass = 0; pass < 2; ++pass) {
-                const uint32_t kb = pass ? skv_lo : skv_hi;
-#pragma unroll 1
-                for (int k = 0; k < D / 16; ++k, ++step) {
-                    const uint64_t ad = t5::desc_sw128(sq_hi + (k >> 2) * PM * 128 + (k & 3) * 32);
-                    const uint64_t bd = t5::desc_sw128(kb + (k >> 2) * PN * 128 + (k & 3) * 32);
-                    t5::mma_f16_ss(t_s, ad, bd, idesc_s, step > 0);
-                }
-            }
-#pragma unroll 1
-            for (int k = 0; k < D / 16; ++k) {
-                const uint64_t bd = t5::desc_sw128(skv_hi + (k >> 2) * PN * 128 + (k & 3) * 32);
-                t5::mma_f16_ts(t_s, t_qlo + 8 * k, bd, idesc_s, true);
-            }
-            t5::mma_commit(mbar);
-        }
-        // ---------------- V~ rows from the staging buffer into registers (during the MMAs)
-        const int vmode = tile_mode(t0, vside);
-        uint32_t xv[64];
-        if (vmode != 0) {
-            const int vfid = vmode == 1 ? vside.fmain.id : vside.ftail.id;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int u = tid + i * PTHREADS;    // (block, g, 8-position group)
-                if (u < NB * 64) {
-                    const int pg = u & 7, g = (u >> 3) & 7, vb = u >> 6;
-                    const uint8_t* rr[8];
-                    uint32_t sel;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) rr[j] = srow(1, t0, t0 + pg + 8 * j, sel);
-                    uint32_t o[4][8];
-                    switch (vfid) {
-                        case F_Q2_0: v_chunk_fast<F_Q2_0, NB>(rr, vb, g, o); break;
-                        case F_Q3_0: v_chunk_fast<F_Q3_0, NB>(rr, vb, g, o); break;
-                        case F_Q4_0: v_chunk_fast<F_Q4_0, NB>(rr, vb, g, o); break;
-                        case F_Q5_0: v_chunk_fast<F_Q5_0, NB>(rr, vb, g, o); break;
-                        case F_Q6_0: v_chunk_fast<F_Q6_0, NB>(rr, vb, g, o); break;
-                        case F_Q8_0: v_chunk_fast<F_Q8_0, NB>(rr, vb, g, o); break;
-                        default: v_chunk_fast<F_F16, NB>(rr, vb, g, o); break;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xv[32 * i + 8 * c + e] = o[c][e];
-                }
-            }
-        } else {
-            const int tg = tid % (PN / 8), cc = tid / (PN / 8);
-            if (cc < CHUNKS) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int t = t0 + tg + 8 * j;
-                    uint32_t sel;
-                    const uint8_t* row = srow(1, t0, t, sel);
-                    Raw8 rv;
-                    fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, rv);
-                    float x[8];
-                    decode_raw8(vside, rv, 8 * cc, x);
-                    const bool live = t <= tile_limit;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) xv[8 * j + e] = __float_as_uint(live ? x[e] : 0.f);
-                }
-            }
-        }
-        // the staging buffer is free: fetch the next tile while this one finishes
-        mma::fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0 && tile + 1 < n_tiles) issue_stage(tile + 1);
-        fault = __syncthreads_or((!mma::mbar_wait(mbar, phase & 1)) || fault) != 0;   // uniform
-        ++phase;
-        t5::fence_after_sync();
-        // ---------------- V~ tile -> V~^T hi/lo (rows = channels, k = positions)
-        if (vmode != 0) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int u = tid + i * PTHREADS;
-                if (u < NB * 64) {
-                    const int pg = u & 7, g = (u >> 3) & 7, vb = u >> 6;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = t5::sw128_offset(32 * vb + 4 * g + c, 8 * pg, D);
-                        const uint32_t* w = &xv[32 * i + 8 * c];
-                        *reinterpret_cast<uint4*>(kv_hi + off) = make_uint4(w[0], w[1], w[2], w[3]);
-                        *reinterpret_cast<uint4*>(kv_lo + off) = make_uint4(w[4], w[5], w[6], w[7]);
-                    }
-                }
-            }
-        } else {
-            const int tg = tid % (PN / 8), cc = tid / (PN / 8);
-            if (cc < CHUNKS) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float y[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) y[j] = __uint_as_float(xv[8 * j + e]);
-                    store_chunk(kv_hi, kv_lo, 8 * cc + e, 8 * tg, D, y);
-                }
-            }
-        }
-        // ---------------- softmax on S (row owners; row-local)
-        if (owner) {
+    if (owner) {
+        // ======================= softmax: S(t) -> P(t), running max and sum of the row
+        for (int t = 0; t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            const int t0 = t * PN;
+            const int sb = t & 1;
+            if (!warp_wait(&s_full[sb], (t >> 1) & 1)) { set_fault(); break; }
+            t5::fence_after_sync();
+            float sv[32];
+            t5::tmem_ld32(t_s + sb * PN + lane_off, sv);
+            t5::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(&s_empty[sb]);
             const bool full = t0 + PN - 1 <= first_row_limit;
             float mx = -INFINITY;
 #pragma unroll
-            for (int hc = 0; hc < PN; hc += 32) {
-                float sv[32];
-                t5::tmem_ld32(t_s + lane_off + hc, sv);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float v = (!full && t0 + slot_pos(hc + i) > my_limit) ? -INFINITY : sv[i];
-                    mx = fmaxf(mx, v);
-                }
+            for (int i = 0; i < PN; ++i) {
+                if (!full && t0 + slot_pos(i) > my_limit) sv[i] = -INFINITY;
+                mx = fmaxf(mx, sv[i]);
             }
             const bool raise = mx > m_run + PF_RESCALE || (m_run == -INFINITY && mx > -INFINITY);
             const float corr = !raise ? 1.f : ((m_run == -INFINITY) ? 0.f : mma::ex2(m_run - mx));
@@ -572,9 +465,14 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 l_run *= corr;
                 m_run = mx;
             }
+            // P and O are read by the previous tile's P V~ MMAs: wait for them
+            if (t > 0) {
+                if (!warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }
+                t5::fence_after_sync();
+            }
             // TMEM loads/stores are warp-collective: rescale O when any lane of the warp
             // raised its max (lanes that did not use factor 1)
-            if (have_o && __any_sync(0xffffffffu, raise)) {
+            if (t > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     float o[32];
@@ -586,55 +484,200 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             }
             float ps = 0.f;
 #pragma unroll
-            for (int hc = 0; hc < PN; hc += 32) {
-                float sv[32];
-                t5::tmem_ld32(t_s + lane_off + hc, sv);
+            for (int i = 0; i < PN; ++i) {
+                const float p = (m_run == -INFINITY || sv[i] == -INFINITY) ? 0.f : mma::ex2(sv[i] - m_run);
+                sv[i] = p;
+                ps += p;
+            }
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool vis = full || t0 + slot_pos(hc + i) <= my_limit;
-                    const float p = (m_run == -INFINITY || !vis) ? 0.f : mma::ex2(sv[i] - m_run);
-                    sv[i] = p;
-                    ps += p;
-                }
+            for (int k0 = 0; k0 < PN; k0 += 8) {
+                float x8[8];
 #pragma unroll
-                for (int k0 = 0; k0 < 32; k0 += 8) {
-                    float x8[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) x8[j] = sv[k0 + j];
-                    store_chunk(p_hi, p_lo, tid, hc + k0, PM, x8);
-                }
+                for (int j = 0; j < 8; ++j) x8[j] = sv[k0 + j];
+                store_chunk64(p_hi, p_lo, tid, k0, x8);
             }
             l_run += ps;
+            t5::fence_proxy_async();
+            t5::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(p_full);
         }
-        t5::fence_proxy_async();
-        t5::fence_before_sync();
-        __syncthreads();
-        t5::fence_after_sync();
-        // ---------------- O += P V~ (3 passes)
-        if (tid == 0) {
-            int step = 0;
-#pragma unroll 1
-            for (int pass = 0; pass < 3; ++pass) {
-                const uint32_t pa = (pass == 2) ? sp_lo : sp_hi;
-                const uint32_t vb = (pass == 1) ? skv_lo : skv_hi;
-#pragma unroll 1
-                for (int k = 0; k < PN / 16; ++k, ++step) {
-                    const uint64_t ad = t5::desc_sw128(pa + (k & 3) * 32);
-                    const uint64_t bd = t5::desc_sw128(vb + (k & 3) * 32);
-                    t5::mma_f16_ss(t_o, ad, bd, idesc_o, have_o || step > 0);
+    } else if (warp < ISSUER_WARP) {
+        // ======================= dequantization: staged rows -> K~(t), V~^T(t)
+        const int dt = tid - 32 * OWNER_WARPS;
+        constexpr int KUNITS = PN * CHUNKS;              // (row, 8-channel chunk)
+        constexpr int VUNITS = (PN / 8) * 8 * NB;        // (8 positions, 4 channels)
+        constexpr int GUNITS = (PN / 8) * CHUNKS * 2;    // generic V: (8 positions, 4 channels)
+        for (int t = 0; t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            const int t0 = t * PN;
+            bool ok = warp_wait(&st_full[t & 1], (t >> 1) & 1);
+            if (ok && t > 0) ok = warp_wait(k_empty, (t - 1) & 1);     // S(t-1) done reading K~
+            if (!ok) { set_fault(); break; }
+            {
+                const int kmode = tile_mode(t0, kside);
+                const int fid = kmode == 1 ? kside.fmain.id : kside.ftail.id;
+                for (int u = dt; u < KUNITS; u += 32 * DQ_WARPS) {
+                    const int kr = u / CHUNKS, ch = u % CHUNKS;
+                    uint32_t sel;
+                    const uint8_t* row = srow(0, t0, t0 + slot_pos(kr), sel);
+                    if (kmode != 0) {
+                        uint32_t out[8];
+                        const int cb = ch >> 2, ct = ch & 3;
+                        switch (fid) {
+                            case F_Q2_0: k_chunk_fast<F_Q2_0, NB>(row, cb, ct, out); break;
+                            case F_Q3_0: k_chunk_fast<F_Q3_0, NB>(row, cb, ct, out); break;
+                            case F_Q4_0: k_chunk_fast<F_Q4_0, NB>(row, cb, ct, out); break;
+                            case F_Q5_0: k_chunk_fast<F_Q5_0, NB>(row, cb, ct, out); break;
+                            case F_Q6_0: k_chunk_fast<F_Q6_0, NB>(row, cb, ct, out); break;
+                            case F_Q8_0: k_chunk_fast<F_Q8_0, NB>(row, cb, ct, out); break;
+                            default: k_chunk_fast<F_F16, NB>(row, cb, ct, out); break;
+                        }
+                        const uint32_t off = t5::sw128_offset(kr, 8 * ch, PN);
+                        *reinterpret_cast<uint4*>(k_hi + off) = make_uint4(out[0], out[1], out[2], out[3]);
+                        *reinterpret_cast<uint4*>(k_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
+                    } else {
+                        Raw8 rk;
+                        fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, rk);
+                        float x[8], y[8];
+                        decode_raw8(kside, rk, 8 * ch, x);
+                        kperm8(x, y);
+                        store_chunk(k_hi, k_lo, kr, 8 * ch, PN, y);
+                    }
                 }
             }
-            t5::mma_commit(mbar);
+            t5::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(k_full);
+            if (t > 0 && !warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }   // P V~(t-1) done reading V~^T
+            const int vmode = tile_mode(t0, vside);
+            if (vmode != 0) {
+                const int vfid = vmode == 1 ? vside.fmain.id : vside.ftail.id;
+                for (int u = dt; u < VUNITS; u += 32 * DQ_WARPS) {
+                    const int pg = u % (PN / 8), g = (u / (PN / 8)) & 7, vb = u / (PN / 8) / 8;
+                    const uint8_t* rr[8];
+                    uint32_t sel;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) rr[j] = srow(1, t0, t0 + pg + (PN / 8) * j, sel);
+                    uint32_t o[4][8];
+                    switch (vfid) {
+                        case F_Q2_0: v_chunk_fast<F_Q2_0, NB>(rr, vb, g, o); break;
+                        case F_Q3_0: v_chunk_fast<F_Q3_0, NB>(rr, vb, g, o); break;
+                        case F_Q4_0: v_chunk_fast<F_Q4_0, NB>(rr, vb, g, o); break;
+                        case F_Q5_0: v_chunk_fast<F_Q5_0, NB>(rr, vb, g, o); break;
+                        case F_Q6_0: v_chunk_fast<F_Q6_0, NB>(rr, vb, g, o); break;
+                        case F_Q8_0: v_chunk_fast<F_Q8_0, NB>(rr, vb, g, o); break;
+                        default: v_chunk_fast<F_F16, NB>(rr, vb, g, o); break;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t off = t5::sw64_offset(32 * vb + 4 * g + c, 8 * pg);
+                        *reinterpret_cast<uint4*>(v_hi + off) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                        *reinterpret_cast<uint4*>(v_lo + off) = make_uint4(o[c][4], o[c][5], o[c][6], o[c][7]);
+                    }
+                }
+            } else {
+                // generic: decode 8 positions x 8 channels, keep one half (4 channels)
+                for (int u = dt; u < GUNITS; u += 32 * DQ_WARPS) {
+                    const int tg = u % (PN / 8), cc = (u / (PN / 8)) % CHUNKS, e4 = u / (PN / 8) / CHUNKS;
+                    float xv[8][4];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int tp = t0 + tg + (PN / 8) * j;
+                        uint32_t sel;
+                        const uint8_t* row = srow(1, t0, tp, sel);
+                        Raw8 rv;
+                        fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, rv);
+                        float x[8];
+                        decode_raw8(vside, rv, 8 * cc, x);
+                        const bool live = tp <= tile_limit;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) xv[j][e] = live ? x[4 * e4 + e] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float y[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) y[j] = xv[j][e];
+                        store_chunk64(v_hi, v_lo, 8 * cc + 4 * e4 + e, 8 * tg, y);
+                    }
+                }
+            }
+            t5::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(v_full);          // also: this tile's staging is consumed
         }
-        fault = __syncthreads_or((!mma::mbar_wait(mbar, phase & 1)) || fault) != 0;   // uniform
-        ++phase;
-        have_o = true;
-        t5::fence_after_sync();
+    } else if (issuer) {
+        // ======================= MMA issue and staging
+        const uint32_t idesc_s = t5::idesc_f16(PM, PN);
+        const uint32_t idesc_o = t5::idesc_f16(PM, D);
+        // descriptors advance by (bytes >> 4) in their start-address field
+        const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
+        const uint64_t dkh0 = t5::desc_sw128(t5::smem_addr(k_hi)), dkl0 = t5::desc_sw128(t5::smem_addr(k_lo));
+        const uint64_t dph0 = t5::desc_sw64(t5::smem_addr(p_hi)), dpl0 = t5::desc_sw64(t5::smem_addr(p_lo));
+        const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(v_hi)), dvl0 = t5::desc_sw64(t5::smem_addr(v_lo));
+        for (int t = 0; t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            const int sb = t & 1;
+            bool ok = mma::mbar_wait(k_full, t & 1);
+            if (ok && t >= 2) ok = mma::mbar_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
+            if (!ok) { set_fault(); break; }
+            t5::fence_after_sync();
+            const uint32_t ts = t_s + sb * PN;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ss(ts, dq0 + dk, dkh0 + dkk, idesc_s, k > 0);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ss(ts, dq0 + dk, dkl0 + dkk, idesc_s, true);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ts(ts, t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
+            }
+            t5::mma_commit(&s_full[sb]);
+            t5::mma_commit(k_empty);
+            s_last = t;
+            ok = mma::mbar_wait(v_full, t & 1);
+            if (ok) ok = mma::mbar_wait(p_full, t & 1);
+            if (!ok) { set_fault(); break; }
+            t5::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dph0 + dk, dvh0 + dk, idesc_o, t > 0 || k > 0);
+            }
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dph0 + dk, dvl0 + dk, idesc_o, true);
+            }
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dpl0 + dk, dvh0 + dk, idesc_o, true);
+            }
+            t5::mma_commit(o_done);
+            o_last = t;
+            if (t + 2 < n_tiles) issue_stage(t + 2);   // this tile's staging buffer is consumed
+        }
     }
 
     // ---- epilogue: O / l -> out (TMEM loads by whole owner warps; only real rows store)
-    const bool any_fault = __syncthreads_or(fault ? 1 : 0) != 0;
-    if (owner && have_o && !any_fault) {
+    __syncthreads();
+    if (owner && !*fault_flag) {
+        if (!warp_wait(o_done, (n_tiles - 1) & 1)) set_fault();
+        t5::fence_after_sync();
+    }
+    __syncthreads();
+    const bool any_fault = *fault_flag != 0;
+    if (owner && !any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         const float inv = row_ok ? 1.f / l_run : 0.f;
 #pragma unroll 1
@@ -652,9 +695,13 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
-    if (any_fault) {
-        // a copy may still be in flight into the staging buffer: give it a bounded wait
-        mma::mbar_wait(sbar, sphase & 1, 100000000ull);
+    if (any_fault && issuer) {
+        // copies and MMAs may still be in flight: give each a bounded wait before the
+        // shared and tensor memory are released
+        for (int i = 0; i < 2; ++i)
+            if (st_last[i] >= 0) mma::mbar_wait(&st_full[i], (st_last[i] >> 1) & 1, 50000000ull);
+        if (s_last >= 0) mma::mbar_wait(&s_full[s_last & 1], (s_last >> 1) & 1, 50000000ull);
+        if (o_last >= 0) mma::mbar_wait(o_done, o_last & 1, 50000000ull);
     }
     t5::fence_before_sync();
     __syncthreads();

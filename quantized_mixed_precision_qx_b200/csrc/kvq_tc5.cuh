@@ -2,7 +2,7 @@
 // (TMEM) allocation, shared-memory matrix descriptors for K-major 128-byte-swizzled fp16
 // operands, the kind::f16 instruction descriptor, MMA issue / commit and TMEM loads.
 //
-// Operand layout used throughout (K-major, SWIZZLE_128B): a tile of R rows x K fp16
+// Main operand layout (K-major, SWIZZLE_128B): a tile of R rows x K fp16
 // elements is stored as K/64 column blocks of R x 128 bytes; inside a column block, rows
 // are grouped in 8-row atoms of 1024 bytes (stride byte offset 1024) and the 16-byte
 // chunk c of row r sits at chunk c ^ (r & 7). An MMA of K = 16 reads 32 bytes of every
@@ -31,6 +31,25 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     d |= (uint64_t)(1024 >> 4) << 32;                // stride byte offset
     d |= (uint64_t)1 << 46;                          // fixed 0b001
     d |= (uint64_t)2 << 61;                          // swizzle mode: 128B
+    return d;
+}
+
+// K-major operand with 64-byte rows (K = 32 fp16), 64B swizzle: element (row, k) at
+// row * 64 + 16 * ((k / 8) ^ ((row / 2) % 4)) + 2 * (k % 8); an MMA step of K = 16 starts
+// 32 bytes further. Tiles start on a 512-byte boundary.
+__device__ __forceinline__ uint32_t sw64_offset(int row, int k) {
+    const int chunk = (k >> 3) ^ ((row >> 1) & 3);
+    return (uint32_t)(row * 64 + chunk * 16 + (k & 7) * 2);
+}
+
+// shared memory matrix descriptor: K-major, 64B swizzle, SBO = 512 bytes (8 rows)
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);          // start address
+    d |= (uint64_t)1 << 16;                          // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(512 >> 4) << 32;                 // stride byte offset
+    d |= (uint64_t)1 << 46;                          // fixed 0b001
+    d |= (uint64_t)4 << 61;                          // swizzle mode: 64B
     return d;
 }
 
