@@ -147,17 +147,28 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
+// With `suspend`, a waiting thread may be suspended by the hardware for up to
+// MBAR_SUSPEND_NS per try (it is woken when the phase completes), so waiting warps leave
+// the issue slots to the others; without it the wait polls (lower wake-up latency).
+constexpr uint32_t MBAR_SUSPEND_NS = 20000;
 // Bounded wait for the phase with parity `parity` to complete. Returns false once about
 // `limit_ns` nanoseconds have passed without completion (the caller records an error and
 // stops waiting), so a wait that can never finish ends the kernel instead of hanging it.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull,
+                                          bool suspend = true) {
     const uint32_t a = smem_u32(bar);
     uint64_t start = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t done;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-            : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        if (suspend) {
+            asm volatile(
+                "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+                : "=r"(done) : "r"(a), "r"(parity), "r"(MBAR_SUSPEND_NS) : "memory");
+        } else {
+            asm volatile(
+                "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+                : "=r"(done) : "r"(a), "r"(parity) : "memory");
+        }
         if (done) return true;
         if ((i & 63) == 0) {
             const uint64_t now = global_ns();

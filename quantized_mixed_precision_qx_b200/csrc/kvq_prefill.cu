@@ -256,7 +256,11 @@ static_assert(PTHREADS == 32 * (ISSUER_WARP + 1), "warp roles");
 
 // bounded wait whose outcome is the same for every lane of the warp
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
-    return __all_sync(0xffffffffu, mma::mbar_wait(bar, parity)) != 0;
+    return __all_sync(0xffffffffu, mma::mbar_wait(bar, parity, 2000000000ull, false)) != 0;
+}
+// the issuer's waits (single thread), polling: they sit on the tensor pipe's critical path
+__device__ __forceinline__ bool poll_wait(uint64_t* bar, uint32_t parity) {
+    return mma::mbar_wait(bar, parity, 2000000000ull, false);
 }
 
 template <int NB>
@@ -619,8 +623,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
             const int sb = t & 1;
-            bool ok = mma::mbar_wait(k_full, t & 1);
-            if (ok && t >= 2) ok = mma::mbar_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
+            bool ok = poll_wait(k_full, t & 1);
+            if (ok && t >= 2) ok = poll_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
             if (!ok) { set_fault(); break; }
             t5::fence_after_sync();
             const uint32_t ts = t_s + sb * PN;
@@ -644,8 +648,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             t5::mma_commit(&s_full[sb]);
             t5::mma_commit(k_empty);
             s_last = t;
-            ok = mma::mbar_wait(v_full, t & 1);
-            if (ok) ok = mma::mbar_wait(p_full, t & 1);
+            ok = poll_wait(v_full, t & 1);
+            if (ok) ok = poll_wait(p_full, t & 1);
             if (!ok) { set_fault(); break; }
             t5::fence_after_sync();
 #pragma unroll
