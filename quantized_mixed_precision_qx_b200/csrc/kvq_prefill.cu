@@ -40,13 +40,18 @@ struct PrefillArgs {
     long long n;                  // cached positions (after the append)
     int C;                        // chunk rows
     int* fault;                   // optional device fault word (may be null)
+    int stage_half;               // bytes of one staging half (PN rows of the widest K|V row), multiple of 16
+    int kbufs;                    // K~ buffers (2 when shared memory allows, else 1)
 };
 
-// raw rows of one tile (K half then V half of a staging buffer): the widest row is 2 D bytes
-__host__ __device__ constexpr size_t stage_half(int D) { return (size_t)PN * 2 * D; }
-__host__ __device__ constexpr size_t pf_smem(int D) {
-    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 4 * stage_half(D) /* 2 staging buffers */ +
-           2 * (size_t)PN * D * 2 /* K~ */ + 2 * (size_t)D * PN * 2 /* V~^T */ + 2 * (size_t)PM * PN * 2 /* P */ + 128 /* barriers */ +
+// shared memory: Q hi, kbufs K~ tiles, V~^T, P (all 1024-byte multiples), then the 2
+// staging buffers of 2 halves (raw K rows, raw V rows of one tile) and the barriers
+__host__ __device__ constexpr size_t pf_tiles(int D, int kbufs) {
+    return (size_t)PM * D * 2 /* Q hi */ + (size_t)kbufs * 2 * PN * D * 2 /* K~ hi, lo */ +
+           2 * (size_t)D * PN * 2 /* V~^T hi, lo */ + 2 * (size_t)PM * PN * 2 /* P hi, lo */;
+}
+__host__ __device__ constexpr size_t pf_smem(int D, int kbufs, size_t stage_half) {
+    return 1024 /* alignment slack */ + pf_tiles(D, kbufs) + 4 * stage_half + 256 /* barriers */ +
            1024 /* tail pad: no operand read can pass the end of the allocation */;
 }
 
@@ -267,29 +272,29 @@ template <int NB>
 __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     constexpr int D = 32 * NB;
     constexpr int CHUNKS = D / 8;                    // 8-channel chunks per row
-    constexpr size_t SH = stage_half(D);
+    const size_t SH = (size_t)a.stage_half;
+    const int KB = a.kbufs;
     const LayerView& lv = a.lv;
     extern __shared__ uint8_t raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* q_hi = sm;                              // Q hi [PM x D]; Q lo lives in TMEM
-    uint8_t* stage = q_hi + PM * D * 2;              // 2 buffers x (K rows, V rows)
-    uint8_t* k_hi = stage + 4 * SH;                  // K~ [PN x D], 128-byte swizzle
-    uint8_t* k_lo = k_hi + PN * D * 2;
-    uint8_t* v_hi = k_lo + PN * D * 2;               // V~^T [D x PN], 64-byte swizzle
+    uint8_t* k_base = q_hi + PM * D * 2;             // K~ [PN x D] hi, lo per buffer, 128-byte swizzle
+    uint8_t* v_hi = k_base + (size_t)KB * 2 * PN * D * 2;   // V~^T [D x PN], 64-byte swizzle
     uint8_t* v_lo = v_hi + D * PN * 2;
     uint8_t* p_hi = v_lo + D * PN * 2;               // P [PM x PN], 64-byte swizzle
     uint8_t* p_lo = p_hi + PM * PN * 2;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);
+    uint8_t* stage = p_lo + PM * PN * 2;             // 2 buffers x (K rows, V rows)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stage + 4 * SH);
     uint64_t* st_full = bars;                        // [2] raw rows of a tile staged
     uint64_t* s_full = bars + 2;                     // [2] S of a tile in TMEM buffer t % 2
     uint64_t* s_empty = bars + 4;                    // [2] owners have read that S buffer
-    uint64_t* k_full = bars + 6;                     // K~ written
-    uint64_t* k_empty = bars + 7;                    // S MMAs done reading K~
-    uint64_t* v_full = bars + 8;                     // V~^T written (and the staging buffer consumed)
-    uint64_t* p_full = bars + 9;                     // P written
-    uint64_t* o_done = bars + 10;                    // P V~ MMAs done
-    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 11);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    uint64_t* k_full = bars + 6;                     // [2] K~ buffer written
+    uint64_t* k_empty = bars + 8;                    // [2] S MMAs done reading that K~ buffer
+    uint64_t* v_full = bars + 10;                    // V~^T written (and the staging buffer consumed)
+    uint64_t* p_full = bars + 11;                    // P written
+    uint64_t* o_done = bars + 12;                    // P V~ MMAs done
+    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 13);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool owner = warp < OWNER_WARPS;           // owns TMEM lane / query row tid
@@ -318,9 +323,9 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             mma::mbar_init(&st_full[i], 1);
             mma::mbar_init(&s_full[i], 1);
             mma::mbar_init(&s_empty[i], OWNER_WARPS);
+            mma::mbar_init(&k_full[i], DQ_WARPS);
+            mma::mbar_init(&k_empty[i], 1);
         }
-        mma::mbar_init(k_full, DQ_WARPS);
-        mma::mbar_init(k_empty, 1);
         mma::mbar_init(v_full, DQ_WARPS);
         mma::mbar_init(p_full, OWNER_WARPS);
         mma::mbar_init(o_done, 1);
@@ -515,8 +520,12 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
             const int t0 = t * PN;
+            // K~ buffer of this tile: free once the S MMAs of tile t - KB have read it
+            const int kb = KB == 2 ? (t & 1) : 0;
+            uint8_t* k_hi = k_base + (size_t)kb * 2 * PN * D * 2;
+            uint8_t* k_lo = k_hi + PN * D * 2;
             bool ok = warp_wait(&st_full[t & 1], (t >> 1) & 1);
-            if (ok && t > 0) ok = warp_wait(k_empty, (t - 1) & 1);     // S(t-1) done reading K~
+            if (ok && t >= KB) ok = warp_wait(&k_empty[kb], (KB == 2 ? (t >> 1) - 1 : t - 1) & 1);
             if (!ok) { set_fault(); break; }
             {
                 const int kmode = tile_mode(t0, kside);
@@ -552,7 +561,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             }
             t5::fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mma::mbar_arrive(k_full);
+            if (lane == 0) mma::mbar_arrive(&k_full[kb]);
             if (t > 0 && !warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }   // P V~(t-1) done reading V~^T
             const int vmode = tile_mode(t0, vside);
             if (vmode != 0) {
@@ -617,15 +626,18 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         const uint32_t idesc_o = t5::idesc_f16(PM, D);
         // descriptors advance by (bytes >> 4) in their start-address field
         const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
-        const uint64_t dkh0 = t5::desc_sw128(t5::smem_addr(k_hi)), dkl0 = t5::desc_sw128(t5::smem_addr(k_lo));
+        const uint64_t dkb0 = t5::desc_sw128(t5::smem_addr(k_base));     // K~ buffer 0, hi part
+        const uint64_t dkstep = (uint64_t)((PN * D * 2) >> 4);             // hi -> lo, and per buffer 2 steps
         const uint64_t dph0 = t5::desc_sw64(t5::smem_addr(p_hi)), dpl0 = t5::desc_sw64(t5::smem_addr(p_lo));
         const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(v_hi)), dvl0 = t5::desc_sw64(t5::smem_addr(v_lo));
-        for (int t = 0; t < n_tiles; ++t) {
-            if (*fault_flag) break;
+        // S MMAs of tile t (waits for K~(t) and for the owners to have read S(t - 2))
+        auto issue_s = [&](int t) -> bool {
             const int sb = t & 1;
-            bool ok = poll_wait(k_full, t & 1);
+            const int kb = KB == 2 ? (t & 1) : 0;
+            const uint64_t dkh0 = dkb0 + (uint64_t)(2 * kb) * dkstep, dkl0 = dkh0 + dkstep;
+            bool ok = poll_wait(&k_full[kb], (KB == 2 ? (t >> 1) : t) & 1);
             if (ok && t >= 2) ok = poll_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
-            if (!ok) { set_fault(); break; }
+            if (!ok) return false;
             t5::fence_after_sync();
             const uint32_t ts = t_s + sb * PN;
 #pragma unroll
@@ -646,11 +658,15 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 t5::mma_f16_ts(ts, t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
             }
             t5::mma_commit(&s_full[sb]);
-            t5::mma_commit(k_empty);
+            t5::mma_commit(&k_empty[kb]);
             s_last = t;
-            ok = poll_wait(v_full, t & 1);
+            return true;
+        };
+        // P V~ MMAs of tile t (waits for V~^T(t) and P(t)), then refill its staging buffer
+        auto issue_pv = [&](int t) -> bool {
+            bool ok = poll_wait(v_full, t & 1);
             if (ok) ok = poll_wait(p_full, t & 1);
-            if (!ok) { set_fault(); break; }
+            if (!ok) return false;
             t5::fence_after_sync();
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
@@ -670,7 +686,17 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             t5::mma_commit(o_done);
             o_last = t;
             if (t + 2 < n_tiles) issue_stage(t + 2);   // this tile's staging buffer is consumed
+            return true;
+        };
+        // S(t) then P V~(t): P V~(t) is queued ahead of S(t + 1) on the tensor pipe, so the
+        // V~^T buffer it reads is released as early as possible
+        bool ok = true;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            ok = issue_s(t);
+            if (ok) ok = issue_pv(t);
         }
+        if (!ok) set_fault();
     }
 
     // ---- epilogue: O / l -> out (TMEM loads by whole owner warps; only real rows store)
@@ -713,11 +739,20 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
 }
 
 template <int NB>
-cudaError_t launch_prefill_nb(const PrefillArgs& a, cudaStream_t st) {
+cudaError_t launch_prefill_nb(PrefillArgs a, cudaStream_t st) {
+    constexpr int D = 32 * NB;
+    // staging halves hold PN rows of the widest row of either side and region
+    int wide = 0;
+    for (int kv = 0; kv < 2; ++kv) {
+        wide = max(wide, a.lv.fmt[kv].stride);
+        if (a.lv.W) wide = max(wide, a.lv.tail.stride);
+    }
+    a.stage_half = PN * wide;
+    a.kbufs = pf_smem(D, 2, (size_t)a.stage_half) <= 227 * 1024 ? 2 : 1;
+    const size_t smem = pf_smem(D, a.kbufs, (size_t)a.stage_half);
     static bool raised = false;
-    const size_t smem = pf_smem(32 * NB);
     if (!raised) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc5<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc5<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         raised = true;
     }
