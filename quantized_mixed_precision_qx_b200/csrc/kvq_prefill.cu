@@ -6,20 +6,23 @@
 // with fp32 accumulators in tensor memory:
 //
 //   CTA   = 128 query rows of one (batch, kv head): row r = chunk row * G + head in group,
-//           TMEM lane r. 16 warps: warps 0-3 own one row per thread (softmax, epilogue);
-//           all share the dequantization.
+//           TMEM lane r. 16 warps in three roles that signal each other through mbarriers:
+//           warps 0-3 own one row per thread (softmax, epilogue), warps 4-14 dequantize,
+//           lane 0 of warp 15 issues the MMAs and the bulk copies.
 //   tile  = 32 key positions. Each tile is dequantized into shared memory as exact fp16
 //           hi + lo parts (K~ = hi + lo; the query and P are split the same way), and
-//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N32 K16 steps) -> TMEM cols [0, 32)
+//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N32 K16 steps) -> TMEM cols [0, 64)
+//               (double-buffered: the softmax reads S(t) while S(t + 1) is written)
 //           O += Ph Vh + Ph Vl + Pl Vh    (3 passes, M128 N=D K16 steps) -> TMEM cols [256, 256 + D)
 //   The softmax is row-local (each thread owns its row), with a lazily raised running max.
-//   K~ and V~^T have buffers of their own, so the P V~ MMAs of a tile run while the next
-//   tile's K~ is dequantized and its S computed; the raw rows of tile i + 1 are fetched by
-//   bulk copies into the second staging buffer while tile i is processed.
+//   K~ (one or two tiles) and V~^T have buffers of their own, so the dequantization of one
+//   tile overlaps the MMAs and the softmax of the previous one; the raw rows of tile t + 2
+//   are fetched by bulk copies into a staging buffer as soon as tile t is dequantized.
 //
-// Shared memory (head_dim D = 32 NB): Q hi 128 x D x 2 B (Q lo lives in TMEM), 2 staging
-// buffers of 2 x 32 raw rows, K~ hi/lo 2 x 32 x D x 2 B (K-major, 128-byte swizzle),
-// V~^T hi/lo 2 x D x 32 x 2 B and P hi/lo 2 x 128 x 32 x 2 B (K-major, 64-byte swizzle).
+// Shared memory (head_dim D = 32 NB): Q hi 128 x D x 2 B (Q lo lives in TMEM), K~ hi/lo
+// 2 x 32 x D x 2 B per K~ tile (K-major, 128-byte swizzle), V~^T hi/lo 2 x D x 32 x 2 B and
+// P hi/lo 2 x 128 x 32 x 2 B (K-major, 64-byte swizzle), 2 staging buffers of 2 x 32 raw rows
+// (sized by the widest row format).
 #include "kvq_internal.cuh"
 #include "kvq_mma.cuh"
 #include "kvq_tc5.cuh"
