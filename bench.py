@@ -312,18 +312,39 @@ def run_kvq(args, rank, world):
     v_host = [c.cpu().pin_memory() for c in v_chunks]
     q_host = q_all.pin_memory()
     out_host = torch.empty(n_steps, B_, HQ_, D_).pin_memory()
-    k_in = torch.empty_like(k_chunks[0])
-    v_in = torch.empty_like(v_chunks[0])
-    q_in = torch.empty(B_, HQ_, D_, device=dev)
+    # inputs are double-buffered on the device and copied on a second stream, so the copy of
+    # step s + 1's inputs overlaps the append and decode of step s (all inside the timing)
+    copy_stream = torch.cuda.Stream(device=dev)
+    k_in = [torch.empty_like(k_chunks[0]) for _ in range(2)]
+    v_in = [torch.empty_like(v_chunks[0]) for _ in range(2)]
+    q_in = [torch.empty(B_, HQ_, D_, device=dev) for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(n_steps)]
+    consumed = [torch.cuda.Event() for _ in range(n_steps)]
+    started = torch.cuda.Event()
+
+    def issue_copy(s):
+        b = s & 1
+        with torch.cuda.stream(copy_stream):
+            if s >= 2:
+                copy_stream.wait_event(consumed[s - 2])      # buffer b is free again
+            k_in[b].copy_(k_host[s], non_blocking=True)
+            v_in[b].copy_(v_host[s], non_blocking=True)
+            q_in[b].copy_(q_host[s], non_blocking=True)
+            copied[s].record(copy_stream)
 
     def e2e_step():
         rebind()
+        started.record(stream)
+        copy_stream.wait_event(started)                      # no copy starts before the step
+        issue_copy(0)
         for s in range(n_steps):
-            k_in.copy_(k_host[s], non_blocking=True)
-            v_in.copy_(v_host[s], non_blocking=True)
-            kvq.kvq_append(h, 0, k_in, v_in, CHUNK, stream)
-            q_in.copy_(q_host[s], non_blocking=True)
-            kvq.kvq_decode_attention(h, 0, q_in, 1.0, out_dev[s], ws, ws.numel(), stream)
+            if s + 1 < n_steps:
+                issue_copy(s + 1)
+            b = s & 1
+            stream.wait_event(copied[s])
+            kvq.kvq_append(h, 0, k_in[b], v_in[b], CHUNK, stream)
+            kvq.kvq_decode_attention(h, 0, q_in[b], 1.0, out_dev[s], ws, ws.numel(), stream)
+            consumed[s].record(stream)
             out_host[s].copy_(out_dev[s], non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
