@@ -10,7 +10,8 @@
 // from the [KVBENCH] cache-size table):
 //   qX_0: d = fp16(absmax / (2^(X-1)-1)) (saturating), q = clamp(rhaz(x / d)), u = q + 2^(X-1)
 //   qX_1: d = fp16((max - min) / (2^X - 1)), m = fp16(min), u = clamp(rhaz((x - m) / d))
-// with IEEE float32 division (__fdiv_rn) and round-half-away-from-zero (roundf).
+// with the IEEE float32 quotient (computed without a division where that is provably
+// identical, see div_range and round_codes) and round-half-away-from-zero (roundf).
 //
 // Ring ([HARDNUM] "KV cache low-bit storage": the last 2,048 positions in an 8-bit ring;
 // [BEELLAMA] precision tail): after an append of C rows to a cache of n, positions
@@ -32,20 +33,44 @@ struct Lanes {
     static constexpr int LPB = 32 / CPL;   // lanes per 32-value block
 };
 
+// fl(1 / (2^k - 1)), k = 0..8 (entry 0 unused)
+__constant__ float c_rcp_range[9] = {0.f, 0x1p+0f, 0x1.555556p-2f, 0x1.24924ap-3f, 0x1.111112p-4f,
+                                     0x1.08421p-5f, 0x1.041042p-6f, 0x1.020408p-7f, 0x1.010102p-8f};
+
+// fl(a / (2^k - 1)) for a >= 0, k = 1..8, without a division: q = fl(a * y) with
+// y = fl(1 / b) is refined once with the exact residual a - q * b (Markstein's division by
+// a constant). Checked exhaustively against IEEE division for every non-negative fp32 a and
+// every b = 2^k - 1 the formats use. An infinite a gives NaN, which the saturating clamp
+// that follows maps to the same value as the quotient inf.
+__device__ __forceinline__ float div_range(float a, int k) {
+    const float b = (float)((1 << k) - 1);
+    const float y = c_rcp_range[k];
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+}
+
+// hardware reciprocal (at most 1 ulp from 1/d)
+__device__ __forceinline__ float rcp_approx(float d) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
+}
+
 constexpr float MAGIC = 12582912.0f;          // 1.5 * 2^23: adding it rounds |r| < 2^22 to an integer
 constexpr int MAGIC_BITS = 0x4B400000;         // bit pattern of MAGIC
 
 // Codes rhaz(fl((x_j - m) / d)) clamped to [lo, hi], for d > 0 (all zero when d == 0), returned as
 // t_j = MAGIC + code (so code = bits(t_j) - MAGIC_BITS and the code as a float is t_j - MAGIC).
-// r = (x - m) * fl(1/d) is within 1.5 * 2^-23 * |r| of fl((x - m) / d). Clamping to integer bounds
-// commutes with rounding, and after it |r| <= lim = max(|lo|, |hi|), so unless r lies within
-// 4e-7 * lim of a half-integer both have the same nearest integer (which is then not a tie) and
-// the rounding add gives it. A lane with such a near-tie redoes its values from the correctly
+// r = (x - m) * rd with rd within 1 ulp of 1/d is within 2 * 2^-23 * |r| of fl((x - m) / d).
+// Clamping to integer bounds commutes with rounding, and after it |r| <= lim = max(|lo|, |hi|),
+// so unless r lies within 4e-7 * lim of a half-integer both have the same nearest integer
+// (which is then not a tie) and the rounding add gives it. A lane with such a near-tie redoes its values from the correctly
 // rounded IEEE quotient, once for all CPL values.
 template <int CPL, bool ASYM>
 __device__ __forceinline__ void round_codes(const float (&x)[CPL], float d, float m, float lo, float hi,
                                             float (&t)[CPL]) {
-    const float rd = d != 0.f ? __frcp_rn(d) : 0.f;
+    const float rd = d != 0.f ? rcp_approx(d) : 0.f;
     const float tol = 4e-7f * fmaxf(-lo, hi);
     bool near = false;
 #pragma unroll
@@ -110,7 +135,7 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
 #pragma unroll
         for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
         a = group_max<LPB>(a);
-        const float d32 = __fdiv_rn(a, (float)qmax);
+        const float d32 = div_range(a, f.bits - 1);      // a / qmax
         dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
         float t[CPL];
@@ -124,7 +149,7 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         for (int j = 1; j < CPL; ++j) { lo = fminf(lo, x[j]); hi = fmaxf(hi, x[j]); }
         lo = group_min<LPB>(lo);
         hi = group_max<LPB>(hi);
-        const float d32 = __fdiv_rn(__fsub_rn(hi, lo), (float)umax);
+        const float d32 = div_range(__fsub_rn(hi, lo), f.bits);   // (hi - lo) / umax
         dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
         mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
@@ -207,7 +232,7 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
 #pragma unroll
             for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
             a = group_max<LPB>(a);
-            const float d32 = __fdiv_rn(a, 127.f);
+            const float d32 = div_range(a, 7);               // a / 127
             const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
             float c[CPL];
             round_codes<CPL, false>(x, d, 0.f, -127.f, 127.f, c);
