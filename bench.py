@@ -518,6 +518,52 @@ def supplementary(dev, peak):
         del c
         torch.cuda.empty_cache()
     res["asymmetric_sweep"] = sweep
+    res["quality_rel_l2_vs_fp32"] = quality(dev)
+    return res
+
+
+FMT_NAMES = ["q2_0", "q2_1", "q3_0", "q3_1", "q4_0", "q4_1", "q5_0", "q5_1", "q6_0", "q6_1", "q8_0", "q8_1"]
+
+
+def quality(dev):
+    """Relative L2 error of the decode output against softmax attention over the unquantized
+    fp32 inputs (computed in float64), per format: K = V = the format, no tail, plus the
+    config D formats with their q8_0 tail. Batch 1, 4 KV heads x 256, 24 query heads, 8192
+    positions with 8 outlier K channels per head (x8), 4 query vectors."""
+    import torch
+    from quantized_mixed_precision_qx_b200 import kvq
+    B, H, Hq, D, n, nq = 1, 4, 24, 256, 8192, 4
+    G = Hq // H
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2024)
+    scale = torch.ones(H, D, device=dev)
+    for h in range(H):
+        scale[h, torch.randperm(D, generator=gen, device=dev)[:8]] = 8.0
+    k = torch.randn(B, n, H, D, device=dev, generator=gen) * scale
+    v = torch.randn(B, n, H, D, device=dev, generator=gen)
+    qs = [torch.randn(B, Hq, D, device=dev, generator=gen) / math.sqrt(D) for _ in range(nq)]
+    # exact reference: query head j reads KV head j // G
+    kk = k.double().permute(0, 2, 1, 3).repeat_interleave(G, dim=1)      # [B][Hq][n][D]
+    vv = v.double().permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    refs = [torch.softmax(torch.einsum("bhd,bhnd->bhn", q.double(), kk), dim=-1).unsqueeze(2).matmul(vv).squeeze(2)
+            for q in qs]
+    cases = [(name, f, f, kvq.NONE, 0) for f, name in enumerate(FMT_NAMES)]
+    cases.append(("q6_0/q5_0 + q8_0 tail 2048", K_FMT, V_FMT, T_FMT, W_))
+    res = {}
+    for name, kf, vf, tf, W in cases:
+        c = kvq.KVCache(1, B, H, Hq, D, n, kf, vf, tf, W, device=dev)
+        for t in range(0, n, 4096):
+            c.append(0, k[:, t:t + 4096].contiguous(), v[:, t:t + 4096].contiguous())
+        ws = c.ensure_workspace(1)
+        num = den = 0.0
+        for q, ref in zip(qs, refs):
+            out = torch.empty_like(q)
+            kvq.kvq_decode_attention(c.handle, 0, q, 1.0, out, ws, ws.numel())
+            torch.cuda.synchronize()
+            num += float(((out.double() - ref) ** 2).sum())
+            den += float((ref ** 2).sum())
+        res[name] = math.sqrt(num / den)
+        del c
     return res
 
 
