@@ -394,10 +394,16 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                             mma_f16(o[j][m], al[m], bp[0][0], bp[0][1]);
                         }
                         if constexpr (VT::asym) {
-                            const float m0 = h2f_lo(reinterpret_cast<const uint16_t*>(vr0 + VT::off_m(NB))[bb]);
-                            const float m1 = h2f_lo(reinterpret_cast<const uint16_t*>(vr1 + VT::off_m(NB))[bb]);
-                            const float m2 = h2f_lo(reinterpret_cast<const uint16_t*>(vr2 + VT::off_m(NB))[bb]);
-                            const float m3 = h2f_lo(reinterpret_cast<const uint16_t*>(vr3 + VT::off_m(NB))[bb]);
+                            // min term of the centred codes: m + d * c (c = (2^bits - 1)/2)
+                            constexpr float VC = VT::vcenter;
+                            const float m0 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr0)[bb]), VC,
+                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr0 + VT::off_m(NB))[bb]));
+                            const float m1 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr1)[bb]), VC,
+                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr1 + VT::off_m(NB))[bb]));
+                            const float m2 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr2)[bb]), VC,
+                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr2 + VT::off_m(NB))[bb]));
+                            const float m3 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr3)[bb]), VC,
+                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr3 + VT::off_m(NB))[bb]));
                             float acc = pm[j];
                             if (v0) acc = fmaf(pv[0], m0, acc);
                             if (v1) acc = fmaf(pv[1], m1, acc);

@@ -23,6 +23,12 @@ struct Fmt {
     static constexpr int w0 = is_float ? 16 : (bits == 8 ? 8 : (bits >= 4 ? 4 : 2));
     static constexpr int w1 = is_float ? 0 : bits - w0;
     static constexpr int off = asym ? 0 : (is_float ? 0 : (1 << (bits - 1)));
+    // V codes enter the P V MMA centred: u - 2^(bits-1) (qX_0) or u - (2^bits - 1)/2 (qX_1, a
+    // half-integer, exact in fp16 for these small codes; the min term then carries
+    // m + d * (2^bits - 1)/2). With all-positive codes the MMA sum and the min term grow large
+    // with opposite signs over long splits, and their cancellation magnifies the accumulation
+    // error of the MMA.
+    static constexpr float vcenter = is_float ? 0.f : (asym ? 0.5f * (float)((1 << bits) - 1) : (float)(1 << (bits - 1)));
     // row byte offsets for nb blocks (see kvq_internal.cuh)
     __device__ static constexpr int off_m(int nb) { return 2 * nb; }
     __device__ static constexpr int off_p0(int nb) { return is_float ? 0 : 2 * nb * (asym ? 2 : 1); }
@@ -189,10 +195,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // 0x6400 is fp16 1024.0: OR-ing a code u < 1024 into the mantissa gives 1024 + u.
 constexpr uint32_t MAGIC = 0x64006400u;
 
-template <int F>
+template <int F, int OFF = Fmt<F>::off>
 __device__ __forceinline__ uint32_t debias(uint32_t x) {
     // (1024 + u) - (1024 + off) = u - off, exact
-    constexpr uint32_t bias_h = 0x6400u + (uint32_t)Fmt<F>::off;   // fp16 bits of 1024 + off (exact, off < 1024)
+    constexpr uint32_t bias_h = 0x6400u + (uint32_t)OFF;   // fp16 bits of 1024 + off (exact, off < 1024)
     const __half2 b = __halves2half2(__ushort_as_half((unsigned short)bias_h), __ushort_as_half((unsigned short)bias_h));
     __half2 v = *reinterpret_cast<__half2*>(&x);
     __half2 r = __hsub2(v, b);
@@ -357,7 +363,16 @@ __device__ __forceinline__ void v_pairs(const uint8_t* ra, const uint8_t* rb, in
             p[3] = and_or(shift<w0 - 3>(y), M, p[3]);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = debias<F>(p[i]);
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (FT::asym) {
+                // (1024 + u) - 1024 = u, then u - c: both exact in fp16
+                const __half2 u2 = *reinterpret_cast<const __half2*>(&p[i]);
+                const __half2 r = __hsub2(__hsub2(u2, __float2half2_rn(1024.f)), __float2half2_rn(FT::vcenter));
+                p[i] = *reinterpret_cast<const uint32_t*>(&r);
+            } else {
+                p[i] = debias<F>(p[i]);
+            }
+        }
     }
 }
 

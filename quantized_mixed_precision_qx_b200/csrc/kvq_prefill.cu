@@ -34,6 +34,10 @@ constexpr int PM = 128;           // query rows per CTA
 constexpr int PN = 32;            // key positions per tile
 constexpr int PTHREADS = 512;     // 16 warps: 4 own the 128 TMEM rows, 11 dequantize, 1 issues
 constexpr float PF_RESCALE = 8.0f;
+// Tiles accumulated into O in tensor memory before the owners fold O into the output row
+// with IEEE fp32 adds and the next P V~ starts a fresh accumulation: long accumulation runs
+// in tensor memory lose precision (over 100k positions the error grows past 1e-4).
+constexpr int PF_FOLD = 64;
 
 struct PrefillArgs {
     LayerView lv;
@@ -449,10 +453,12 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     auto set_fault = [&]() { *fault_flag = 1; };
 
     float m_run = -INFINITY, l_run = 0.f;
+    float gcorr = 1.f;                               // owners: pending rescale of the folded partial
     int s_last = -1, o_last = -1;                    // issuer: last tile whose S / P V~ MMAs were committed
 
     if (owner) {
         // ======================= softmax: S(t) -> P(t), running max and sum of the row
+        float* const orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
             const int t0 = t * PN;
@@ -482,16 +488,41 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                 if (!warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }
                 t5::fence_after_sync();
             }
-            // TMEM loads/stores are warp-collective: rescale O when any lane of the warp
-            // raised its max (lanes that did not use factor 1)
-            if (t > 0 && __any_sync(0xffffffffu, raise)) {
+            if (t > 0 && t % PF_FOLD == 0) {
+                // fold: O in TMEM holds tiles [t - PF_FOLD, t); add it to the partial in the
+                // output row, apply this tile's correction; P V~(t) then starts afresh
+                const bool first = t == PF_FOLD;
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     float o[32];
-                    t5::tmem_ld32(t_o + lane_off + c, o);
+                    t5::tmem_ld32(t_o + lane_off + c, o);      // warp-collective
+                    if (row_ok) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= corr;
-                    t5::tmem_st32(t_o + lane_off + c, o);
+                        for (int i = 0; i < 32; i += 4) {
+                            float4 g4 = first ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                              : *reinterpret_cast<const float4*>(orow + c + i);
+                            g4.x = (g4.x * gcorr + o[i]) * corr;
+                            g4.y = (g4.y * gcorr + o[i + 1]) * corr;
+                            g4.z = (g4.z * gcorr + o[i + 2]) * corr;
+                            g4.w = (g4.w * gcorr + o[i + 3]) * corr;
+                            *reinterpret_cast<float4*>(orow + c + i) = g4;
+                        }
+                    }
+                }
+                gcorr = 1.f;
+            } else {
+                gcorr *= corr;                           // the folded partial follows the max lazily
+                // TMEM loads/stores are warp-collective: rescale O when any lane of the warp
+                // raised its max (lanes that did not use factor 1)
+                if (t > 0 && __any_sync(0xffffffffu, raise)) {
+#pragma unroll 1
+                    for (int c = 0; c < D; c += 32) {
+                        float o[32];
+                        t5::tmem_ld32(t_o + lane_off + c, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= corr;
+                        t5::tmem_st32(t_o + lane_off + c, o);
+                    }
                 }
             }
             float ps = 0.f;
@@ -674,7 +705,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
                 const uint64_t dk = (uint64_t)((k * 32) >> 4);
-                t5::mma_f16_ss(t_o, dph0 + dk, dvh0 + dk, idesc_o, t > 0 || k > 0);
+                t5::mma_f16_ss(t_o, dph0 + dk, dvh0 + dk, idesc_o, t % PF_FOLD != 0 || k > 0);
             }
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
@@ -713,15 +744,21 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     if (owner && !any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         const float inv = row_ok ? 1.f / l_run : 0.f;
+        const bool folded = n_tiles > PF_FOLD;      // a partial of earlier tiles is in orow
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
             float o[32];
             t5::tmem_ld32(t_o + lane_off + c, o);
             if (row_ok) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4*>(orow + c + i) =
-                        make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+                for (int i = 0; i < 32; i += 4) {
+                    float4 g4 = folded ? *reinterpret_cast<const float4*>(orow + c + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    g4.x = (g4.x * gcorr + o[i]) * inv;
+                    g4.y = (g4.y * gcorr + o[i + 1]) * inv;
+                    g4.z = (g4.z * gcorr + o[i + 2]) * inv;
+                    g4.w = (g4.w * gcorr + o[i + 3]) * inv;
+                    *reinterpret_cast<float4*>(orow + c + i) = g4;
+                }
             }
         }
     } else if (row_ok && any_fault) {
