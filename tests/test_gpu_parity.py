@@ -213,3 +213,21 @@ def test_append_half_step_ties(tail, W):
         g.append(0, torch.from_numpy(x).cuda(), torch.from_numpy(x).cuda())
         o.append(0, x, x)
         compare_bytes(g, o, 0, 1, H, T, W)
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_multi_query_chunks(D):
+    """Multi-query verification (a few draft tokens appended, then attended causally): chunks
+    of 1, 2 and 8 rows through the prefill entry point, the window boundary inside the cache."""
+    W = 96
+    wl = Workload(1, 1, 2, 12, D, 1200, KVRecipe("outlier"), seed=60)
+    g, o = make_pair(wl, orc.Q6_0, orc.Q5_0, orc.Q8_0, W)
+    vmax = append_both(g, o, wl, 0, 0, 1189)
+    t = 1189
+    for cid, C in enumerate([1, 2, 8]):
+        vmax = max(vmax, append_both(g, o, wl, 0, t, t + C))
+        t += C
+        q = wl.q_prefill(0, C, chunk_id=cid)
+        out = g.prefill(0, to_dev(q), 1.0).cpu().numpy()
+        ref = o.prefill(0, q, 1.0)
+        check_close(out, ref, vmax, f"multi-query C={C} D={D}")
