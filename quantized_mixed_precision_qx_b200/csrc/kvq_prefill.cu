@@ -37,7 +37,7 @@ constexpr float PF_RESCALE = 8.0f;
 // Tiles accumulated into O in tensor memory before the owners fold O into the output row
 // with IEEE fp32 adds and the next P V~ starts a fresh accumulation: long accumulation runs
 // in tensor memory lose precision (over 100k positions the error grows past 1e-4).
-constexpr int PF_FOLD = 64;
+constexpr int PF_FOLD = 128;
 
 struct PrefillArgs {
     LayerView lv;
