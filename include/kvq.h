@@ -55,7 +55,8 @@ typedef enum kvq_status {
     KVQ_ERR_EMPTY = 5,           /* attention over an empty cache */
     KVQ_ERR_ALIGNMENT = 6,       /* a device pointer is not 16-byte aligned */
     KVQ_ERR_NOT_BOUND = 7,       /* no device buffer bound yet */
-    KVQ_ERR_CUDA = 8             /* a CUDA runtime call or launch failed */
+    KVQ_ERR_CUDA = 8,            /* a CUDA runtime call or launch failed */
+    KVQ_ERR_DEVICE_TIMEOUT = 9   /* a kernel gave up a bounded device-side wait (see kvq_device_status) */
 } kvq_status;
 
 /* Block formats. A block is 32 consecutive channels of one token row ([HARDNUM],
@@ -103,20 +104,31 @@ typedef struct kvq_cache kvq_cache;
 KVQ_API kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_fmt,
                             kvq_fmt tail_fmt, int32_t W, kvq_cache** out);
 
-/* Bytes of device memory the cache needs: the low-bit store (max_ctx rows per layer,
- * batch element, kv head, K and V), the ring (W rows each) and the KVarN scales. Equal
- * to the block-size closed form when every row is a multiple of 16 bytes and max_ctx,
- * W are multiples of 16 (rows are otherwise padded to 16 bytes, regions to 256). */
+/* Bytes of device memory the cache needs ([BEELLAMA] KV-MiB table and [KVBENCH] cache-size
+ * column: the store is max_ctx rows of the block format per layer, kv head, K and V; the
+ * precision tail adds W rows of the tail format on top): the low-bit store, the ring, the
+ * KVarN scales and a metadata region of 256 + 16 * n_layers * batch * n_kv_heads bytes
+ * rounded up to 256 (a device status word and per-head value bounds). Without the
+ * metadata region this equals the block-size closed form when every row is a multiple of
+ * 16 bytes and max_ctx, W are multiples of 16 (rows are otherwise padded to 16 bytes,
+ * regions to 256). */
 KVQ_API kvq_status kvq_cache_required_bytes(const kvq_cache* cache, size_t* bytes);
 
 /* Bind caller-owned device memory (>= required bytes, 256-byte aligned) on the current
- * device. Zero-fills it on `stream` and resets every layer's length to 0. */
+ * device: the memory holds the rows [OFFLOAD] sizes per token and layer (row-size
+ * paragraph) in the block formats above. Zero-fills it on `stream` and resets every
+ * layer's length to 0. Also maps the fixed array of kvq_decode_attention_noalloc on this
+ * device (looked up once per device). KVQ_ERR_CUDA if a CUDA call fails. */
 KVQ_API kvq_status kvq_cache_bind(kvq_cache* cache, void* dev_buf, size_t bytes, void* stream);
 
-/* Free the host descriptor (never the bound device memory). NULL is accepted. */
+/* Free the host descriptor (never the bound device memory). NULL is accepted. Nothing on
+ * the pages corresponds to it; it ends the descriptor's lifetime. */
 KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
 
-/* Quantize-on-append of n_new positions to layer `layer` (all batch elements).
+/* Quantize-on-append of n_new positions to layer `layer` (all batch elements)
+ * ([HARDNUM] "Reddit reactions": each token row is quantized in 32-value blocks as it
+ * enters, and blocks are requantized when the window boundary moves; "KV cache low-bit
+ * storage": the last 2,048 positions stay in the 8-bit ring).
  * k, v: float32 [batch][n_new][n_kv_heads][head_dim]. Positions n..n+n_new-1 are
  * written: those that end inside the window go to the ring in tail format (evicting
  * and requantizing the positions they displace), the others straight to the low-bit
@@ -128,10 +140,15 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const float* k, c
                       int32_t n_new, void* stream);
 
 /* Workspace bytes for kvq_decode_attention (n_query_rows = 1) or kvq_prefill_attention
- * (n_query_rows = n_chunk). The workspace holds per-split softmax partials. */
+ * (n_query_rows = n_chunk). The workspace holds the per-split softmax partials of the
+ * split-K decode ([OFFLOAD]: decode streams the whole attention state each step, so the
+ * positions are split across the GPU and the partials merged). KVQ_ERR_NOT_BOUND before a
+ * bind (the split count depends on the device's SM count). */
 KVQ_API kvq_status kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t n_query_rows, size_t* bytes);
 
-/* Decode attention (GQA) over all n cached positions of `layer`:
+/* Decode attention (GQA) over all n cached positions of `layer` ([OFFLOAD] decode-is-
+ * bandwidth paragraph: each step reads every cached row; [HARDNUM] "KV cache low-bit
+ * storage": the low-bit rows plus the 8-bit recent-token ring of config D):
  * out[b][hq] = softmax_t(scale * q[b][hq] . K~[b][hq/G][t]) . V~[b][hq/G][t], with K~, V~
  * the dequantized cache (ring rows for the last min(n, W) positions). q, out: float32
  * [batch][n_q_heads][head_dim]. Split-K over positions, then a fixed-order merge, so the
@@ -140,9 +157,10 @@ KVQ_API kvq_status kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t n_
 KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const float* q, float scale,
                                 float* out, void* ws, size_t ws_bytes, void* stream);
 
-/* Causal chunked-prefill attention for the n_chunk positions just appended: chunk row i
+/* Causal chunked-prefill attention for the n_chunk positions just appended ([HARDNUM]
+ * "Engine speed and cache reuse": prompt processing with the config D cache; chunk row i
  * sits at position n - n_chunk + i and attends to positions <= its own over the
- * post-append cache. q, out: float32 [batch][n_chunk][n_q_heads][head_dim].
+ * post-append cache). q, out: float32 [batch][n_chunk][n_q_heads][head_dim].
  * Requires 1 <= n_chunk <= n. ws: >= kvq_decode_workspace_bytes(n_chunk). */
 KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const float* q, int32_t n_chunk,
                                  float scale, float* out, void* ws, size_t ws_bytes, void* stream);
@@ -154,8 +172,10 @@ KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const 
  * owns the device allocator, or a C caller whose device footprint must stay fixed after
  * start-up). The pages have no counterpart to this entry point; it is a deployment aid.
  *  - Every GPU that loads the library holds the array until the process exits.
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *    with the cache's device current; make that first call before any stream capture.
+ *  - The array's device address is looked up (cudaGetSymbolAddress) once per device, when
+ *    a cache is first bound on it (kvq_cache_bind) or at the first call on it, with that
+ *    device current; with CUDA's lazy module loading that lookup is also when the array
+ *    is mapped. Make that first bind or call before any stream capture.
  *  - The cache's device must be the current device (KVQ_ERR_INVALID_ARG otherwise).
  *  - A cache whose decode needs more workspace than the array holds
  *    (kvq_decode_workspace_bytes(cache, 1) > KVQ_NOALLOC_WORKSPACE_MIB MiB) is rejected
@@ -168,15 +188,39 @@ KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const 
 KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const float* q, float scale,
                                         float* out, void* stream);
 
-/* Current number of cached positions of `layer` (host-tracked, uniform over batch). */
+/* Current number of cached positions of `layer` (host-tracked, uniform over batch): the
+ * context length n of [HARDNUM] "KV cache low-bit storage", which decides which positions
+ * are in the recent-token ring (the last min(n, W)). */
 KVQ_API kvq_status kvq_length(const kvq_cache* cache, int32_t layer, int64_t* n);
 
-/* KVarN only: set the channel scales of `layer` instead of calibrating. sK, sV: device
- * float32 [batch][n_kv_heads][head_dim], all > 0. Must come before the layer's first append. */
+/* KVarN only ([BEELLAMA] KVarN paragraph: variance-normalised blocks): set the channel
+ * scales of `layer` instead of calibrating. sK, sV: device float32
+ * [batch][n_kv_heads][head_dim], all > 0. Must come before the layer's first append. */
 KVQ_API kvq_status kvq_set_channel_scales(kvq_cache* cache, int32_t layer, const float* sK, const float* sV,
                                   void* stream);
 
-/* Copy stored rows to host memory in the canonical serialisation (per 32-value block:
+/* KVarN only ([BEELLAMA] KVarN paragraph): copy the channel scales of `layer` (calibrated
+ * or set) to host memory. host_sK, host_sV: float32 [batch][n_kv_heads][head_dim].
+ * Synchronises the device. KVQ_ERR_CALIBRATION if the layer has no scales yet. */
+KVQ_API kvq_status kvq_get_channel_scales(const kvq_cache* cache, int32_t layer, float* host_sK, float* host_sV);
+
+/* Device status of the cache. Every wait a kernel makes on the device (a pipeline barrier)
+ * is bounded; a wait that runs out makes the kernel stop waiting, poison its output with NaN
+ * and record the event in a status word inside the bound buffer. This call synchronises
+ * `stream`, reads the word and clears it: KVQ_OK if no wait ran out since the last call,
+ * KVQ_ERR_DEVICE_TIMEOUT otherwise. The pages have no counterpart; it is the failure
+ * report of the pipelined kernels. */
+KVQ_API kvq_status kvq_device_status(kvq_cache* cache, void* stream);
+
+/* Check of the failure path above: one warp waits, with the same bounded wait the
+ * pipelined kernels use and a limit of limit_ns (<= 10 s), on a barrier that nothing
+ * arrives on, then records the timeout in the cache's status word (kvq_device_status then
+ * returns KVQ_ERR_DEVICE_TIMEOUT). Holds no copies or tensor memory. Asynchronous on
+ * `stream`. The pages have no counterpart. */
+KVQ_API kvq_status kvq_selftest_wait_timeout(kvq_cache* cache, uint64_t limit_ns, void* stream);
+
+/* Copy stored rows to host memory in the canonical serialisation of [KVBENCH] /
+ * [BEELLAMA] block byte counts (per 32-value block:
  * fp16 d | [fp16 m] | code planes low bits first, little endian; BF16/F16: 32 x 2 bytes).
  * region 0: low-bit store rows pos0..pos0+count-1; region 1: ring slots pos0..+count-1
  * (tail format). kv: 0 = K, 1 = V. Synchronises the device. host_dst must hold
@@ -184,7 +228,7 @@ KVQ_API kvq_status kvq_set_channel_scales(kvq_cache* cache, int32_t layer, const
 KVQ_API kvq_status kvq_export_blocks(const kvq_cache* cache, int32_t layer, int32_t b, int32_t h, int32_t kv,
                              int32_t region, int64_t pos0, int64_t count, void* host_dst, size_t bytes);
 
-/* Static description of a status code. */
+/* Static description of a status code (no counterpart on the pages). */
 KVQ_API const char* kvq_status_string(kvq_status status);
 
 #ifdef __cplusplus

@@ -104,11 +104,16 @@ __device__ __forceinline__ void pack_store(uint8_t* p0, uint8_t* p1, int lane, c
 }
 
 // Quantize this lane's CPL values into row `row` of format f (all lanes participate).
+// Returns an upper bound of |stored value| over this lane's values (the block bound d*qmax,
+// or |m| + d*umax, for block formats; the 16-bit rounding of |x| for bf16 / f16 rows).
 template <int CPL>
-__device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFmt& f, int lane,
-                                          const float (&x)[CPL]) {
+__device__ __forceinline__ float store_row(uint8_t* __restrict__ row, const RowFmt& f, int lane,
+                                           const float (&x)[CPL]) {
     constexpr int LPB = Lanes<CPL>::LPB;
     if (f.kind != 0) {
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
         uint16_t h[CPL];
 #pragma unroll
         for (int j = 0; j < CPL; ++j)
@@ -124,11 +129,12 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
 #pragma unroll
             for (int j = 0; j < CPL; ++j) dst[j] = h[j];
         }
-        return;
+        return a * 1.0078125f;          // a 16-bit rounding grows |x| by at most 2^-8
     }
     const int blk = (lane * CPL) >> 5;
     uint32_t u[CPL];
     uint16_t dh, mh = 0;
+    float bound;
     if (!f.asym) {
         const int qmax = (1 << (f.bits - 1)) - 1;
         float a = 0.f;
@@ -138,6 +144,7 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         const float d32 = div_range(a, f.bits - 1);      // a / qmax
         dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
+        bound = d * (float)qmax;
         float t[CPL];
         round_codes<CPL, false>(x, d, 0.f, (float)-qmax, (float)qmax, t);
 #pragma unroll
@@ -154,6 +161,7 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
         const float d = __half2float(__ushort_as_half(dh));
         const float m = __half2float(__ushort_as_half(mh));
+        bound = fabsf(m) + d * (float)umax;
         float t[CPL];
         round_codes<CPL, true>(x, d, m, 0.f, (float)umax, t);
 #pragma unroll
@@ -173,17 +181,49 @@ __device__ __forceinline__ void store_row(uint8_t* __restrict__ row, const RowFm
         reinterpret_cast<uint16_t*>(row)[blk] = dh;
         if (f.asym) reinterpret_cast<uint16_t*>(row + f.off_m)[blk] = mh;
     }
+    return bound;
 }
+
+// Value bounds of the rows a warp stores: stored domain (block values) and dequantized
+// domain (after the KVarN channel scale).
+struct Bounds {
+    float stored = 0.f, deq = 0.f;
+    __device__ void add(float s, float d) { stored = fmaxf(stored, s); deq = fmaxf(deq, d); }
+};
 
 // Low-bit store of a raw row (KVarN: divide by the channel scales first).
 template <int CPL>
 __device__ __forceinline__ void store_low(uint8_t* row, const RowFmt& f, const float* __restrict__ s, int lane,
-                                          float (&x)[CPL]) {
+                                          float (&x)[CPL], Bounds& bd) {
+    float smax = 1.f;
     if (s) {
+        smax = 0.f;
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) x[j] = __fdiv_rn(x[j], s[lane * CPL + j]);
+        for (int j = 0; j < CPL; ++j) {
+            const float sc = s[lane * CPL + j];
+            smax = fmaxf(smax, sc);
+            x[j] = __fdiv_rn(x[j], sc);
+        }
     }
-    store_row<CPL>(row, f, lane, x);
+    const float b = store_row<CPL>(row, f, lane, x);
+    bd.add(b, b * smax);
+}
+
+// Raise the cache's per-head bounds (float bits of non-negative values compare as unsigned
+// integers) to this warp's; the read first keeps the atomic off the common path.
+__device__ __forceinline__ void publish_bounds(uint32_t* st, Bounds bd) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        bd.stored = fmaxf(bd.stored, __shfl_xor_sync(0xffffffffu, bd.stored, off));
+        bd.deq = fmaxf(bd.deq, __shfl_xor_sync(0xffffffffu, bd.deq, off));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        // margin for the fp32 rounding of dequantized values
+        const uint32_t u0 = __float_as_uint(bd.stored * 1.0009765625f);
+        const uint32_t u1 = __float_as_uint(bd.deq * 1.0009765625f);
+        if (u0 > __ldcg(st)) atomicMax(st, u0);
+        if (u1 > __ldcg(st + 1)) atomicMax(st + 1, u1);
+    }
 }
 
 template <int CPL>
@@ -207,11 +247,14 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     const float* s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * D : nullptr;
     const uint32_t p = n + i;
 
+    uint32_t* st = lv.stats + ((long long)(b * lv.H + h) * 2 + kv) * 2;
+    Bounds bd;
     float x[CPL];
     load_row_f32<CPL>(src, lane, x);
 
     if (lv.W == 0) {
-        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, x);
+        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, x, bd);
+        publish_bounds(st, bd);
         return;
     }
     const uint32_t W = (uint32_t)lv.W;
@@ -239,7 +282,8 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
 #pragma unroll
             for (int j = 0; j < CPL; ++j) t[j] = __fmul_rn(d, __fsub_rn(c[j], MAGIC));
         }
-        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, t);
+        store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, t, bd);
+        publish_bounds(st, bd);
         return;
     }
     // ends inside the window: evict the slot's old occupant, then take the slot
@@ -253,10 +297,12 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
         float y[CPL];
         load_row_values<CPL>(srow, lv.tail, lane, y);
         __syncwarp();
-        store_low<CPL>(main + (long long)q * fl.stride, fl, s, lane, y);
+        store_low<CPL>(main + (long long)q * fl.stride, fl, s, lane, y, bd);
     }
     __syncwarp();
-    store_row<CPL>(srow, lv.tail, lane, x);
+    const float rb = store_row<CPL>(srow, lv.tail, lane, x);   // ring rows hold raw values
+    bd.add(rb, rb);
+    publish_bounds(st, bd);
 }
 
 // KVarN statistics: one CTA of T/2 threads per (b, h, K|V, channel group of 8);

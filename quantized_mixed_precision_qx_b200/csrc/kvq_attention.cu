@@ -246,7 +246,25 @@ cudaError_t run_pass1(const P1Args& a, int n_region_split, int B, cudaStream_t s
     return cudaGetLastError();
 }
 
+// One warp waits, with the pipelines' bounded wait, on an mbarrier that nothing arrives on;
+// the wait runs out after limit_ns and the timeout is recorded like a pipeline's would be.
+__global__ void wait_selftest(uint32_t* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mma::mbar_init(&bar, 1);
+        mma::fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = __all_sync(0xffffffffu, mma::mbar_wait(&bar, 0, limit_ns, false)) != 0;
+    if (!ok && threadIdx.x == 0) atomicOr(status, STATUS_WAIT_TIMEOUT);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t st) {
+    wait_selftest<<<1, 32, 0, st>>>(status, limit_ns);
+    return cudaGetLastError();
+}
 
 size_t partial_floats(int G, int D) { return (size_t)G * (D + 2); }
 
@@ -329,6 +347,8 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
             t.q = q;
             t.qscale = a.qscale;
             t.scales = lv.kvarn ? lv.scales : nullptr;
+            t.stats = lv.stats;
+            t.status = lv.status;
             t.ws = ws;
             t.n = n;
             t.pos_base = a.pos_base;

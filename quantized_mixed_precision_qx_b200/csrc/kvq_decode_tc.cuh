@@ -41,6 +41,8 @@ struct Args {
     const float* q;         // [B][rows][Hq][D]
     float qscale;           // scale * log2(e)
     const float* scales;    // KVarN [B][H][2][D] or nullptr
+    const uint32_t* stats;  // the layer's value bounds [B][H][2][2] (float bits)
+    uint32_t* status;       // device status word (a timed-out wait is recorded here)
     float* ws;
     long long n;            // cached positions
     long long pos_base;     // position of query row 0
@@ -73,9 +75,12 @@ constexpr size_t XS_BYTES = 2 * CWARPS * 32 * sizeof(float4);       // double-bu
 __host__ __device__ constexpr int query_parts(int kf) { return kf == F_BF16 ? 3 : 2; }
 __host__ __device__ constexpr size_t qs_bytes(int parts) { return (size_t)NBMAX * 2 * parts * 32 * sizeof(uint2); }
 constexpr size_t QSUM_BYTES = NBMAX * 8 * sizeof(float);
+constexpr size_t QEXP_BYTES = 2 * 8 * sizeof(float);     // per head: 2^-e (query scaling), 2^e (score)
 __host__ __device__ constexpr size_t smem_bytes(int ks, int vs, int D, int parts) {
-    return main_bytes(ks, vs, D) + PT_BYTES + XS_BYTES + qs_bytes(parts) + QSUM_BYTES + 2 * STAGES * sizeof(uint64_t) + 16;
+    return main_bytes(ks, vs, D) + PT_BYTES + XS_BYTES + qs_bytes(parts) + QSUM_BYTES + QEXP_BYTES +
+           2 * STAGES * sizeof(uint64_t) + 16;
 }
+
 
 // OR of `pred` over the 64 threads of a warp pair (named barrier `id`); also orders the
 // pair's shared-memory accesses like bar.sync
@@ -112,7 +117,8 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     float4* xs = reinterpret_cast<float4*>(smem + mb + PT_BYTES);                      // [2][CWARPS][32]
     uint2* qs = reinterpret_cast<uint2*>(smem + mb + PT_BYTES + XS_BYTES);             // [NB][2][KP][32]
     float* qsum_s = reinterpret_cast<float*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP));   // [NB][8]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP) + QSUM_BYTES);
+    float* qexp_s = qsum_s + NBMAX * 8;                                                  // [2][8]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP) + QSUM_BYTES + QEXP_BYTES);
     uint64_t* empty = full + STAGES;
     int* fault = reinterpret_cast<int*>(empty + STAGES);
 
@@ -136,6 +142,15 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     const int kvarn = a.scales != nullptr && !a.ring;
     const float* sK = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 0) * D : nullptr;
     const float* sV = kvarn ? a.scales + ((long long)(b * H + h) * 2 + 1) * D : nullptr;
+
+    // V block values enter the MMA folded as fp16 hi + lo of d * c: scale d by 2^-ev so that
+    // every |d * c| of the cache (bounded by the stats the appends keep) stays below 2^15, or
+    // up into fp16's normal range for tiny caches
+    int ev = 0;
+    if constexpr (!VT::is_float) ev = fp16_exponent(__uint_as_float(a.stats[((long long)(b * H + h) * 2 + 1) * 2]), -10, 9);
+    const float vexp = __uint_as_float((uint32_t)(127 + ev) << 23);         // 2^ev
+    const __half vm1 = __float2half_rn(__uint_as_float((uint32_t)(127 - ev) << 23));
+    const uint32_t vmul = (uint32_t)__half_as_ushort(vm1) * 0x10001u;       // 2^-ev in both halves
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // query values of this lane's fragments (warp w builds block w), loaded first so their
@@ -173,6 +188,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     // ------------------------------------------------------------ producer warp
     if (warp == CWARPS) {
         if (lane == 0) {
+            int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
                 const int s = it % STAGES;
                 if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) { *fault = 1; break; }
@@ -183,14 +199,45 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                 mbar_arrive_expect_tx(&full[s], kb + vb);
                 bulk_g2s(st, kreg + r0 * a.kstride, kb, &full[s]);
                 bulk_g2s(st + (size_t)TOK * a.kstride, vreg + r0 * a.vstride, vb, &full[s]);
+                issued = it + 1;
+            }
+            // before the stages are reused for the final combine (or the CTA exits), every
+            // copy issued must have landed: wait (bounded) for the last tile of each stage;
+            // when the consumers saw every tile this returns at once
+            for (int s = 0; s < STAGES; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % STAGES + STAGES) % STAGES;
+                if (issued > s && last >= 0) mbar_wait(&full[s], (last / STAGES) & 1, 50000000ull);
             }
         }
     }
 
     // ------------------------------------------------------------ query fragments
-    // (B operand of QK, head g of lane (g, t)), built while the first tiles are in flight
+    // (B operand of QK, head g of lane (g, t)), built while the first tiles are in flight.
+    // Each head's scaled query is normalised by a power of two 2^-e (e = 0 unless it lies
+    // outside the fp16-friendly range); its scores are multiplied back by 2^e.
     if (warp < CWARPS) {
+        {
+            const int hh = warp;                     // CWARPS == 8 heads
+            float mq = 0.f;
+            if (hh < G) {
+                const float* qh = a.q + ((long long)br * G * H + (long long)h * G + hh) * D;
+                for (int c = lane; c < D; c += 32) {
+                    float x = qh[c] * a.qscale;
+                    if (kvarn) x *= sK[c];
+                    mq = fmaxf(mq, fabsf(x));
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, off));
+            if (lane == 0) {
+                const int e = fp16_exponent(mq, -100, 100);
+                qexp_s[hh] = __uint_as_float((uint32_t)(127 - e) << 23);
+                qexp_s[8 + hh] = __uint_as_float((uint32_t)(127 + e) << 23);
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * CWARPS) : "memory");
+        }
         if (warp < NB) {
+            const float qn = qexp_s[g];
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 float v[4];
@@ -198,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                 for (int sl = 0; sl < 4; ++sl) {
                     float x = qv[m][sl] * a.qscale;
                     if (kvarn) x *= sK[32 * warp + q_channel<KF>(t, m, sl)];
-                    v[sl] = x;
+                    v[sl] = x * qn;
                 }
                 uint32_t p01[3], p23[3];
                 split_pack<KF>(v[0], v[1], p01);
@@ -214,10 +261,11 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                 float sacc = 0.f;
                 if (hh < G) {
                     const float* qh = a.q + ((long long)br * G * H + (long long)h * G + hh) * D + 32 * bb;
+                    const float qn = qexp_s[hh];
                     for (int c = 0; c < 32; ++c) {
                         float x = qh[c] * a.qscale;
                         if (kvarn) x *= sK[32 * bb + c];
-                        sacc += x;
+                        sacc += x * qn;
                     }
                 }
                 qsum_s[idx] = sacc;
@@ -247,6 +295,8 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
         const long long W = a.W;
         const long long nmodw = a.ring ? a.n % W : 0;
         const int sub0 = 16 * tg;
+        const float qe0 = qexp_s[8 + 2 * t], qe1 = qexp_s[8 + 2 * t + 1];   // 2^e of heads 2t, 2t+1
+        const bool qscaled = qe0 != 1.f || qe1 != 1.f;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % STAGES;
             const bool ok = mbar_wait(&full[s], (it / STAGES) & 1);
@@ -312,6 +362,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                     const float4 ps = xb[(warp ^ TGROUPS) * 32 + lane];
                     sc[0] += ps.x; sc[1] += ps.y; sc[2] += ps.z; sc[3] += ps.w;   // commutative: same in both
                 }
+                if (qscaled) { sc[0] *= qe0; sc[1] *= qe1; sc[2] *= qe0; sc[3] *= qe1; }
                 if (!valid(g)) { sc[0] = -INFINITY; sc[1] = -INFINITY; }
                 if (!valid(g + 8)) { sc[2] = -INFINITY; sc[3] = -INFINITY; }
                 // ---------------- online softmax for heads 2t, 2t+1
@@ -386,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                     const int bb = b0 + j;
                     if constexpr (VSCALED) {
                         uint32_t ah[2][4], al[2][4];
-                        v_frags_scaled<VF>(vr0, vr1, vr2, vr3, NB, bb, g, ah, al);
+                        v_frags_scaled<VF>(vr0, vr1, vr2, vr3, NB, bb, g, vmul, ah, al);
 #pragma unroll
                         for (int m = 0; m < 2; ++m) {
                             mma_f16(o[j][m], ah[m], bp[0][0], bp[0][1]);
@@ -498,6 +549,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
         cM[hh] = M;
         cL[hh] = bad ? __int_as_float(0x7fc00000) : L;   // a timed-out wait poisons the result
     }
+    if (bad && threadIdx.x == 0) atomicOr(a.status, STATUS_WAIT_TIMEOUT);
     __syncthreads();
     float* part = a.ws + ((((long long)br * H + h) * a.n_split) + a.split_offset + split) * ((long long)G * (D + 2));
     // o = sum over row groups of weight * o_w, two channels per thread step (8-byte stores)
@@ -510,8 +562,11 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
             float2 ow = *reinterpret_cast<const float2*>(&co[(w * 8 + hh) * D + c]);
             if constexpr (VT::asym) {
                 const float pmw = cpm[(w * 8 + hh) * NBMAX + (c >> 5)];
-                ow.x += pmw;
-                ow.y += pmw;
+                ow.x = fmaf(ow.x, vexp, pmw);
+                ow.y = fmaf(ow.y, vexp, pmw);
+            } else if constexpr (VSCALED) {
+                ow.x *= vexp;
+                ow.y *= vexp;
             }
             o0 = fmaf(ow.x, e, o0);
             o1 = fmaf(ow.y, e, o1);

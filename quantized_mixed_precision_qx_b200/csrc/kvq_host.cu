@@ -17,7 +17,7 @@ struct kvq_cache {
     int kf, vf, tf, W;
     RowFmt fmt[2], tail;
     // byte offsets of the areas inside the bound buffer
-    size_t off_main[2], off_ring[2], off_scales;
+    size_t off_main[2], off_ring[2], off_scales, off_meta;
     size_t main_region[2], ring_region;   // bytes per (layer, b, h) region
     size_t total;
     uint8_t* buf;
@@ -30,6 +30,13 @@ struct kvq_cache {
 namespace {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// metadata region: a 256-byte header (word 0 = device status) and 4 uint32 value bounds per
+// (layer, batch element, kv head)
+constexpr size_t META_HEADER_WORDS = 64;
+size_t meta_bytes(const kvq_layout& L) {
+    return align_up(META_HEADER_WORDS * 4 + (size_t)L.n_layers * L.batch * L.n_kv_heads * 4 * sizeof(uint32_t), 256);
+}
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
@@ -48,6 +55,9 @@ LayerView layer_view(const kvq_cache* c, int layer) {
                                 (size_t)layer * units * 2 * c->L.head_dim
                           : nullptr;
     v.tail = c->tail;
+    uint32_t* meta = reinterpret_cast<uint32_t*>(c->buf + c->off_meta);
+    v.status = meta;
+    v.stats = meta + META_HEADER_WORDS + (size_t)layer * units * 4;
     v.B = c->L.batch;
     v.H = c->L.n_kv_heads;
     v.D = c->L.head_dim;
@@ -58,6 +68,9 @@ LayerView layer_view(const kvq_cache* c, int layer) {
 }
 
 kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+// device address of the no-allocation workspace on `dev` (defined with the entry point below)
+kvq_status noalloc_workspace(int dev, void** ptr);
 
 }  // namespace
 
@@ -74,6 +87,7 @@ const char* kvq_status_string(kvq_status s) {
         case KVQ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
         case KVQ_ERR_NOT_BOUND: return "no device buffer bound";
         case KVQ_ERR_CUDA: return "CUDA error";
+        case KVQ_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait on the device ran out";
     }
     return "unknown status";
 }
@@ -122,6 +136,8 @@ kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_f
     }
     c->off_scales = off;
     if (L.kvarn) off += align_up(units * 2 * D * sizeof(float), 256);
+    c->off_meta = off;
+    off += meta_bytes(L);
     c->total = off;
     c->buf = nullptr;
     c->buf_bytes = 0;
@@ -147,6 +163,11 @@ kvq_status kvq_cache_bind(kvq_cache* c, void* dev_buf, size_t bytes, void* strea
     if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemsetAsync(dev_buf, 0, c->total, (cudaStream_t)stream) != cudaSuccess) return KVQ_ERR_CUDA;
+    // map the no-allocation entry point's fixed array now, while the caller is setting up,
+    // rather than at its first call (lazy module loading maps it at the first lookup)
+    void* ws = nullptr;
+    kvq_status s = noalloc_workspace(dev, &ws);
+    if (s != KVQ_OK) return s;
     c->buf = (uint8_t*)dev_buf;
     c->buf_bytes = bytes;
     c->device = dev;
@@ -182,6 +203,41 @@ kvq_status kvq_set_channel_scales(kvq_cache* c, int32_t layer, const float* sK, 
         return KVQ_ERR_CUDA;
     c->scales_set[layer] = 1;
     return KVQ_OK;
+}
+
+kvq_status kvq_get_channel_scales(const kvq_cache* c, int32_t layer, float* host_sK, float* host_sV) {
+    if (!c || !host_sK || !host_sV || layer < 0 || layer >= c->L.n_layers || !c->L.kvarn) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    if (!c->scales_set[layer]) return KVQ_ERR_CALIBRATION;
+    const LayerView v = layer_view(c, layer);
+    const size_t row = (size_t)c->L.head_dim * sizeof(float);
+    const int BH = c->L.batch * c->L.n_kv_heads;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemcpy2D(host_sK, row, v.scales, 2 * row, row, BH, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy2D(host_sV, row, (const uint8_t*)v.scales + row, 2 * row, row, BH, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    return KVQ_OK;
+}
+
+kvq_status kvq_device_status(kvq_cache* c, void* stream) {
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t* word = reinterpret_cast<uint32_t*>(c->buf + c->off_meta);
+    uint32_t h = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemcpy(&h, word, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (h == 0) return KVQ_OK;
+    if (cudaMemsetAsync(word, 0, sizeof(uint32_t), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    return KVQ_ERR_DEVICE_TIMEOUT;
+}
+
+kvq_status kvq_selftest_wait_timeout(kvq_cache* c, uint64_t limit_ns, void* stream) {
+    if (!c || limit_ns > 10000000000ull) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    uint32_t* word = reinterpret_cast<uint32_t*>(c->buf + c->off_meta);
+    return cuda_status(launch_wait_selftest(word, (unsigned long long)limit_ns, (cudaStream_t)stream));
 }
 
 kvq_status kvq_append(kvq_cache* c, int32_t layer, const float* k, const float* v, int32_t n_new, void* stream) {
@@ -324,8 +380,8 @@ kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32
 // The array lives in this library's device image: every GPU on which the library is
 // loaded holds its KVQ_NOALLOC_WS_BYTES until the process exits. In host code its name
 // only stands for the device symbol; the device address is looked up once per device
-// with cudaGetSymbolAddress (on the entry point's first call on that device, with that
-// device current) and cached. Every call shares the array and it keeps the last call's
+// with cudaGetSymbolAddress (when a cache is first bound on that device, or at the entry
+// point's first call there, with that device current) and cached. Every call shares the array and it keeps the last call's
 // contents; the decode's first pass writes every partial the merge reads, so nothing has
 // to start at zero. Calls whose kernels overlap on the GPU (several streams, several
 // threads) race on the array.

@@ -7,6 +7,12 @@
 //   K ring  [L][B][H] regions of W rows (tail format row stride)        (W > 0)
 //   V ring  [L][B][H] regions of W rows                                  (W > 0)
 //   scales  [L][B][H][2][D] float32 KVarN channel scales                 (kvarn)
+//   meta    256-byte header (word 0: device status, bits set by a kernel whose bounded
+//           wait ran out) then stats [L][B][H][2 (K|V)][2] uint32: float bits of upper
+//           bounds of |value| over every row stored so far, [0] in the stored domain
+//           (the block values d*c (+m), before the KVarN channel scale) and [1] in the
+//           dequantized domain (after it). Kernels use them to pick power-of-two scalings
+//           that keep 16-bit tensor-core operands inside the fp16 range.
 // A low-bit row of D channels (nb = D/32 blocks) is stored as
 //   [d: nb x fp16][m: nb x fp16, qX_1 only][plane0: D*w0/8 bytes][plane1: D*w1/8 bytes]
 // padded to 16 bytes. Each plane is the little-endian bitstream of the row's codes in
@@ -84,9 +90,33 @@ struct LayerView {
     long long ring_region; // bytes per (b, h) ring region
     RowFmt fmt[2];         // K / V low-bit formats
     RowFmt tail;           // tail format (kind 0 = q8_0)
+    uint32_t* stats;       // this layer's [B][H][2][2] value bounds (see the layout above)
+    uint32_t* status;      // the cache's device status word
     int B, H, D, G, W;
     int kvarn;
 };
+
+// device status bits
+constexpr uint32_t STATUS_WAIT_TIMEOUT = 1u;
+
+// Power-of-two exponent e such that bound * 2^-e < 2^15 with bound * 2^-e >= 2^14 (0 for a
+// zero or non-finite bound), clamped to [lo, hi].
+__host__ __device__ inline int pow2_exponent(float bound, int lo, int hi) {
+    if (!(bound > 0.f) || !(bound < 3.0e38f)) return 0;
+    int e = 0;
+    (void)frexpf(bound, &e);       // bound = f * 2^e, f in [0.5, 1)
+    e -= 15;
+    return e < lo ? lo : (e > hi ? hi : e);
+}
+
+// Scaling for 16-bit tensor-core operands: a value range whose maximum m already lies in
+// [2^-4, 2^14) is left alone (exponent 0); otherwise m * 2^-e lands in [2^14, 2^15), inside
+// fp16's range with the normal-range precision of its hi + lo split for all but values
+// 2^18 times smaller than m.
+__host__ __device__ inline int fp16_exponent(float m, int lo, int hi) {
+    if (m >= 0.0625f && m < 16384.f) return 0;
+    return pow2_exponent(m, lo, hi);
+}
 
 // ---------------------------------------------------------------- launches
 cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
@@ -120,5 +150,9 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
 bool prefill_supported(int D);
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
                            cudaStream_t st);
+
+// One warp waits, with the bounded wait the pipelined kernels use and a limit of limit_ns,
+// on an mbarrier that nothing ever arrives on, then records the timeout in *status.
+cudaError_t launch_wait_selftest(uint32_t* status, unsigned long long limit_ns, cudaStream_t st);
 
 }  // namespace kvq

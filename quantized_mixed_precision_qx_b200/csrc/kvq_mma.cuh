@@ -397,17 +397,21 @@ __device__ __forceinline__ void v_frags(const uint8_t* r0, const uint8_t* r1, co
 // (r0, r1) and (r2, r3), x = d * (u - off) is computed in fp16 as hi = RN(d * c) and the
 // exact remainder lo = d * c - hi (fused multiply-add, single rounding; d * c has at most
 // 17 significant bits, so hi + lo == d * c unless the fp16 subnormal range is reached).
+// vmul: a power of two 2^-e in both fp16 halves, applied to the scales first (exact while
+// d * 2^-e stays representable) so that every d * c of the cache fits fp16; the caller
+// multiplies the accumulated output by 2^e.
 template <int F>
 __device__ __forceinline__ void v_frags_scaled(const uint8_t* r0, const uint8_t* r1, const uint8_t* r2,
-                                               const uint8_t* r3, int nb, int b, int g,
+                                               const uint8_t* r3, int nb, int b, int g, uint32_t vmul,
                                                uint32_t (&ahi)[2][4], uint32_t (&alo)[2][4]) {
     uint32_t pa[4], pb[4];
     v_pairs<F>(r0, r1, nb, b, g, pa);
     v_pairs<F>(r2, r3, nb, b, g, pb);
     const uint32_t d01 = prmt(reinterpret_cast<const uint16_t*>(r0)[b], reinterpret_cast<const uint16_t*>(r1)[b], 0x5410u);
     const uint32_t d23 = prmt(reinterpret_cast<const uint16_t*>(r2)[b], reinterpret_cast<const uint16_t*>(r3)[b], 0x5410u);
-    const __half2 da = *reinterpret_cast<const __half2*>(&d01);
-    const __half2 db = *reinterpret_cast<const __half2*>(&d23);
+    const __half2 vm = *reinterpret_cast<const __half2*>(&vmul);
+    const __half2 da = __hmul2_rn(*reinterpret_cast<const __half2*>(&d01), vm);
+    const __half2 db = __hmul2_rn(*reinterpret_cast<const __half2*>(&d23), vm);
     uint32_t ha[4], la[4], hb[4], lb[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

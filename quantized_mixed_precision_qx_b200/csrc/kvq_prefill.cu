@@ -11,7 +11,8 @@
 //           lane 0 of warp 15 issues the MMAs and the bulk copies.
 //   tile  = 32 key positions. Each tile is dequantized into shared memory as exact fp16
 //           hi + lo parts (K~ = hi + lo; the query and P are split the same way), and
-//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N32 K16 steps) -> TMEM cols [0, 64)
+//           S = Qh Kh^T + Qh Kl^T + Ql Kh^T (3 passes, M128 N32 K16 steps) -> TMEM cols [0, 128)
+//               (two partial sums over the channel halves, added by the softmax warps)
 //               (double-buffered: the softmax reads S(t) while S(t + 1) is written)
 //           O += Ph Vh + Ph Vl + Pl Vh    (3 passes, M128 N=D K16 steps) -> TMEM cols [256, 256 + D)
 //   The softmax is row-local (each thread owns its row), with a lazily raised running max.
@@ -46,7 +47,6 @@ struct PrefillArgs {
     float qscale;                 // scale * log2(e)
     long long n;                  // cached positions (after the append)
     int C;                        // chunk rows
-    int* fault;                   // optional device fault word (may be null)
     int stage_half;               // bytes of one staging half (PN rows of the widest K|V row), multiple of 16
     int kbufs;                    // K~ buffers (2 when shared memory allows, else 1)
 };
@@ -324,6 +324,13 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     const int W = lv.W;
     const int ring0 = W > 0 ? n - W : n;             // first position held in the ring
     const int n_tiles = tile_limit / PN + 1;
+    // K~ and V~ enter the MMAs scaled by 2^-ek, 2^-ev (exponents from the bounds the appends
+    // keep, 0 for ordinary ranges) so that their fp16 hi + lo parts neither overflow nor lose
+    // their low part to fp16's subnormal range; S and O are scaled back exactly
+    const int ek = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 0) * 2 + 1]), -120, 120);
+    const int ev = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 1) * 2 + 1]), -120, 120);
+    const float kmul = __uint_as_float((uint32_t)(127 - ek) << 23);
+    const float vmul = __uint_as_float((uint32_t)(127 - ev) << 23);
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -344,8 +351,12 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem;                       // S: columns [0, PN) and [PN, 2 PN)
-    const uint32_t t_qlo = tmem + 64;                // Q lo: columns [64, 64 + D/2)
+    // S of buffer sb: two partial sums over the channel halves (columns 2 PN sb + [0, PN) and
+    // 2 PN sb + [PN, 2 PN)), added with IEEE fp32 adds by the owners: the tensor-memory
+    // accumulation then runs over half the k-steps, which halves its rounding error at
+    // large logits
+    const uint32_t t_s = tmem;                       // S: columns [0, 4 PN)
+    const uint32_t t_qlo = tmem + 4 * PN;            // Q lo: columns [4 PN, 4 PN + D/2)
     const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
 
@@ -392,9 +403,23 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         if (n_tiles > 1) issue_stage(1);
     }
 
-    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row)
+    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row). A row
+    // is normalised by a power of two 2^-eq (eq = 0 for ordinary ranges); its scores are
+    // multiplied back by 2^(eq + ek).
+    float s_mul = 1.f;
     if (owner) {
         const float* qr = a.q + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        float qn = 1.f;
+        if (row_ok) {
+            float mq = 0.f;
+            for (int c = 0; c < D; c += 4) {
+                const float4 p = *reinterpret_cast<const float4*>(qr + c);
+                mq = fmaxf(mq, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(p.z), fabsf(p.w))));
+            }
+            const int eq = fp16_exponent(mq * fabsf(a.qscale), -120, 120);
+            qn = __uint_as_float((uint32_t)(127 - eq) << 23);
+            s_mul = __uint_as_float((uint32_t)(127 + eq) << 23) * __uint_as_float((uint32_t)(127 + ek) << 23);
+        }
 #pragma unroll 1
         for (int c64 = 0; c64 < D; c64 += 64) {      // 64 k-values = 32 TMEM columns
             float cols[32];
@@ -406,7 +431,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                     const float4 v = *reinterpret_cast<const float4*>(qr + c64 + k0 + 4);
                     x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w; x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) x[j] *= a.qscale;
+                    for (int j = 0; j < 8; ++j) x[j] = (x[j] * a.qscale) * qn;
                 } else {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) x[j] = 0.f;
@@ -432,7 +457,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     // Tile modes (uniform over the CTA): 1 = every position in the low-bit store and its
     // format has a fast path, 2 = every position in the ring with a fast tail format,
     // 0 = generic decode (mixed tiles, asymmetric / bf16 formats, KVarN).
-    auto tile_mode = [&](int t0, const SideView& v) -> int {
+    auto tile_mode = [&](int t0, const SideView& v, int e) -> int {
+        if (e != 0) return 0;                        // scaled values take the generic path
         const int last = min(t0 + PN - 1, tile_limit);
         if (last < ring0 && !v.scales && fast_fmt(v.fmain.id)) return 1;
         if (t0 >= ring0 && fast_fmt(v.ftail.id)) return 2;
@@ -465,11 +491,18 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             const int sb = t & 1;
             if (!warp_wait(&s_full[sb], (t >> 1) & 1)) { set_fault(); break; }
             t5::fence_after_sync();
-            float sv[32];
-            t5::tmem_ld32(t_s + sb * PN + lane_off, sv);
+            float sv[32], sv2[32];
+            t5::tmem_ld32(t_s + 2 * PN * sb + lane_off, sv);
+            t5::tmem_ld32(t_s + 2 * PN * sb + PN + lane_off, sv2);
             t5::fence_before_sync();
             __syncwarp();
             if (lane == 0) mma::mbar_arrive(&s_empty[sb]);
+#pragma unroll
+            for (int i = 0; i < PN; ++i) sv[i] += sv2[i];
+            if (s_mul != 1.f) {
+#pragma unroll
+                for (int i = 0; i < PN; ++i) sv[i] *= s_mul;
+            }
             const bool full = t0 + PN - 1 <= first_row_limit;
             float mx = -INFINITY;
 #pragma unroll
@@ -562,7 +595,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             if (ok && t >= KB) ok = warp_wait(&k_empty[kb], (KB == 2 ? (t >> 1) - 1 : t - 1) & 1);
             if (!ok) { set_fault(); break; }
             {
-                const int kmode = tile_mode(t0, kside);
+                const int kmode = tile_mode(t0, kside, ek);
                 const int fid = kmode == 1 ? kside.fmain.id : kside.ftail.id;
                 for (int u = dt; u < KUNITS; u += 32 * DQ_WARPS) {
                     const int kr = u / CHUNKS, ch = u % CHUNKS;
@@ -588,6 +621,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                         fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, rk);
                         float x[8], y[8];
                         decode_raw8(kside, rk, 8 * ch, x);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) x[j] *= kmul;
                         kperm8(x, y);
                         store_chunk(k_hi, k_lo, kr, 8 * ch, PN, y);
                     }
@@ -597,7 +632,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             __syncwarp();
             if (lane == 0) mma::mbar_arrive(&k_full[kb]);
             if (t > 0 && !warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }   // P V~(t-1) done reading V~^T
-            const int vmode = tile_mode(t0, vside);
+            const int vmode = tile_mode(t0, vside, ev);
             if (vmode != 0) {
                 const int vfid = vmode == 1 ? vside.fmain.id : vside.ftail.id;
                 for (int u = dt; u < VUNITS; u += 32 * DQ_WARPS) {
@@ -639,7 +674,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                         decode_raw8(vside, rv, 8 * cc, x);
                         const bool live = tp <= tile_limit;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) xv[j][e] = live ? x[4 * e4 + e] : 0.f;
+                        for (int e = 0; e < 4; ++e) xv[j][e] = live ? x[4 * e4 + e] * vmul : 0.f;
                     }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -673,23 +708,24 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             if (ok && t >= 2) ok = poll_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
             if (!ok) return false;
             t5::fence_after_sync();
-            const uint32_t ts = t_s + sb * PN;
+            const uint32_t ts = t_s + 2 * PN * sb;
+            constexpr int KH = D / 32;                 // k-steps per channel half
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
                 const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ss(ts, dq0 + dk, dkh0 + dkk, idesc_s, k > 0);
+                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkh0 + dkk, idesc_s, (k % KH) > 0);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
                 const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ss(ts, dq0 + dk, dkl0 + dkk, idesc_s, true);
+                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkl0 + dkk, idesc_s, true);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ts(ts, t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
+                t5::mma_f16_ts(ts + (k >= KH ? PN : 0), t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
             }
             t5::mma_commit(&s_full[sb]);
             t5::mma_commit(&k_empty[kb]);
@@ -743,7 +779,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     const bool any_fault = *fault_flag != 0;
     if (owner && !any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
-        const float inv = row_ok ? 1.f / l_run : 0.f;
+        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_run : 0.f;
         const bool folded = n_tiles > PF_FOLD;      // a partial of earlier tiles is in orow
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
@@ -762,6 +798,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
             }
         }
     } else if (row_ok && any_fault) {
+        if (tid == 0) atomicOr(lv.status, STATUS_WAIT_TIMEOUT);
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
@@ -814,7 +851,6 @@ cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, flo
     a.qscale = scale * 1.4426950408889634f;
     a.n = n;
     a.C = C;
-    a.fault = nullptr;
     if (lv.D == 256) return launch_prefill_nb<8>(a, st);
     if (lv.D == 128) return launch_prefill_nb<4>(a, st);
     return cudaErrorInvalidValue;

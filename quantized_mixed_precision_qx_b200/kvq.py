@@ -21,12 +21,13 @@ FMT_NAMES = ["q2_0", "q2_1", "q3_0", "q3_1", "q4_0", "q4_1", "q5_0", "q5_1",
 
 # status codes (kvq_status)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_FMT, ERR_CAPACITY, ERR_CALIBRATION, ERR_EMPTY, \
-    ERR_ALIGNMENT, ERR_NOT_BOUND, ERR_CUDA = range(9)
+    ERR_ALIGNMENT, ERR_NOT_BOUND, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(10)
 
 EXPORTED = ["kvq_cache_create", "kvq_cache_required_bytes", "kvq_cache_bind", "kvq_cache_destroy",
             "kvq_append", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_prefill_attention",
             "kvq_length", "kvq_set_channel_scales", "kvq_export_blocks", "kvq_status_string",
-            "kvq_decode_attention_noalloc"]
+            "kvq_decode_attention_noalloc", "kvq_get_channel_scales", "kvq_device_status",
+            "kvq_selftest_wait_timeout"]
 NOALLOC_WORKSPACE_BYTES = 8 << 20     # KVQ_NOALLOC_WORKSPACE_MIB
 
 
@@ -66,6 +67,9 @@ def lib():
             "kvq_decode_attention_noalloc": [p, i32, p, f32, p, p],
             "kvq_length": [p, i32, ctypes.POINTER(i64)],
             "kvq_set_channel_scales": [p, i32, p, p, p],
+            "kvq_get_channel_scales": [p, i32, p, p],
+            "kvq_device_status": [p, p],
+            "kvq_selftest_wait_timeout": [p, ctypes.c_uint64, p],
             "kvq_export_blocks": [p, i32, i32, i32, i32, i32, i64, i64, p, sz],
         }
         for name, args in sigs.items():
@@ -157,6 +161,21 @@ def kvq_set_channel_scales(cache, layer: int, sK, sV, stream=None):
            "kvq_set_channel_scales")
 
 
+def kvq_get_channel_scales(cache, layer: int, host_sK, host_sV):
+    """host_sK, host_sV: writable float32 numpy arrays [batch][n_kv_heads][head_dim]."""
+    _check(lib().kvq_get_channel_scales(cache, layer, ctypes.c_void_p(host_sK.ctypes.data),
+                                        ctypes.c_void_p(host_sV.ctypes.data)), "kvq_get_channel_scales")
+
+
+def kvq_device_status(cache, stream=None) -> int:
+    """Status code (OK or ERR_DEVICE_TIMEOUT) of the cache's device status word; clears it."""
+    return lib().kvq_device_status(cache, _stream(stream))
+
+
+def kvq_selftest_wait_timeout(cache, limit_ns: int, stream=None):
+    _check(lib().kvq_selftest_wait_timeout(cache, limit_ns, _stream(stream)), "kvq_selftest_wait_timeout")
+
+
 def kvq_export_blocks(cache, layer: int, b: int, h: int, kv: int, region: int, pos0: int, count: int,
                       host_dst) -> None:
     """host_dst: a writable numpy uint8 array."""
@@ -222,6 +241,13 @@ class KVCache:
 
     def set_channel_scales(self, layer, sK, sV, stream=None):
         kvq_set_channel_scales(self.handle, layer, sK, sV, stream)
+
+    def channel_scales(self, layer):
+        import numpy as np
+        sK = np.empty((self.B, self.H, self.D), dtype=np.float32)
+        sV = np.empty_like(sK)
+        kvq_get_channel_scales(self.handle, layer, sK, sV)
+        return sK, sV
 
     def row_bytes(self, region, kv):
         f = self.tail_fmt if region == 1 else (self.v_fmt if kv else self.k_fmt)
