@@ -1,6 +1,7 @@
-"""Algorithmic byte accounting of the benchmark (the numerators of every GB/s and roofline
-fraction it reports), against closed forms of the block layout: K q6_0 rows of 208 B, V
-q5_0 rows of 176 B and q8_0 ring rows of 272 B at head_dim 256, fp32 inputs."""
+"""Algorithmic byte and FLOP accounting of the benchmark (the numerators of every GB/s,
+TFLOP/s and roofline fraction it reports), against closed forms of the block layout: K q6_0
+rows of 208 B, V q5_0 rows of 176 B and q8_0 ring rows of 272 B at head_dim 256, fp32
+inputs; and the causal prefill FLOP count of the full-length workload."""
 import os
 import sys
 
@@ -36,3 +37,34 @@ def test_append_bytes_filling_and_bulk():
     assert bench.append_bytes(65536, 8192) == 4 * (8192 * 2048 + 2048 * 544 * 2 + 8192 * 384)
     # no ring
     assert bench.append_bytes(0, 100, W=0) == 4 * 100 * (2048 + 384)
+
+
+def test_headline_step_accounting():
+    a = bench.step_accounting()
+    # 64 decode steps x 16 layers at 262,081 .. 262,144: 4 KV heads x ((n - 2048) x 384 + 2048 x 544) + q, out
+    want = 16 * sum(4 * ((n - 2048) * 384 + 2048 * 544) + 2 * 24 * 256 * 4 for n in range(262081, 262145))
+    assert a["decode_bytes"] == want
+    # one decode at 262,080 reads ~404 MB (399.5 MB of low-bit rows + 4.46 MB of ring rows)
+    assert abs(bench.decode_bytes(262080) - 403.9e6) < 0.1e6
+    # the fill: 257,984 positions per layer; the first 2,048 only touch the ring, every later
+    # position is written once to the low-bit store; 2,048 stay in the ring at the end
+    per_layer = 4 * (257984 * 2048 + (257984 - 2048) * 384 + 2048 * 544 + (32 - 1) * 2048 * 544 * 2)
+    assert a["fill_bytes"] == 16 * per_layer
+    assert a["fill_positions"] == 16 * 257984
+    # launches: 32 fill appends + the chunk append + the prefill per layer; each decode step
+    # appends once and launches the ring pass, the low-bit pass and the merge per layer
+    assert a["launches"] == 16 * 34 + 16 * 64 * 4
+
+
+def test_prefill_flop_count():
+    # row i of the 4,096-row chunk attends to 257,984 + i + 1 keys: sum = C n + C (C + 1) / 2
+    keys = 4096 * 257984 + 4096 * 4097 // 2
+    assert bench.prefill_flops(257984, 4096) == keys * 24 * 4 * 256
+    assert abs(bench.prefill_flops(257984, 4096) - 2.62e13) < 0.01e13      # per layer
+    assert bench.prefill_flops(0, 1) == 24 * 4 * 256
+
+
+def test_end_to_end_copy_volumes():
+    # every fill append's K and V, the chunk's K, V and queries, the decode steps' K, V, q
+    assert bench.hi_h2d() == 16 * 4 * (257984 * 2 * 4 * 256 + 4096 * (2 * 4 * 256 + 24 * 256) + 64 * (2 * 4 * 256 + 24 * 256))
+    assert bench.hi_d2h() == 16 * 4 * (4096 + 64) * 24 * 256
