@@ -66,6 +66,7 @@ def lib():
             "orc_export": (c_i, [c_p, c_i, c_i, c_i, c_i, c_i, c_i64, c_i64, c_p]),
             "orc_position_row": (c_i, [c_p, c_i, c_i, c_i, c_i, c_i64, c_p]),
             "orc_decode": (c_i, [c_p, c_i, c_p, c_f, c_p, c_i]),
+            "orc_decode_indexed": (c_i, [c_p, c_i, c_p, c_f, c_p, c_i, c_p, c_i]),
             "orc_prefill": (c_i, [c_p, c_i, c_p, c_i, c_f, c_p, c_p, c_i, c_i]),
         }
         for name, (res, args) in sig.items():
@@ -221,6 +222,16 @@ class Cache:
         assert q.shape == (self.B, self.Hq, self.D)
         out = np.zeros_like(q)
         self._chk(lib().orc_decode(self._h, layer, _ptr(q), scale, _ptr(out), self.threads), "decode")
+        return out
+
+    def decode_indexed(self, layer, q, idx, scale=1.0):
+        """Decode over the positions listed per (batch, kv head): idx int32 [B][H][k]."""
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        assert q.shape == (self.B, self.Hq, self.D) and idx.shape[:2] == (self.B, self.H)
+        out = np.zeros_like(q)
+        self._chk(lib().orc_decode_indexed(self._h, layer, _ptr(q), scale, _ptr(idx), idx.shape[2], _ptr(out),
+                                           self.threads), "decode_indexed")
         return out
 
     def prefill(self, layer, q, scale=1.0, rows=None):

@@ -461,6 +461,49 @@ void attend_rows(const Cache& C, int l, int b, int h, int64_t n, int64_t t_end,
         for (int c = 0; c < D; ++c) outs[g][c] = (float)(o[(size_t)g * D + c] / den[g]);
 }
 
+// Softmax attention of one query row (all G heads of kv head h) over an explicit list of
+// positions (the index-gather decode: [OFFLOAD], the paragraph on the QSA indexer choosing a
+// budget of 2,048 positions per step). READING: entries outside [0, n) are skipped; the
+// others enter in list order, a repeated position counting once per entry; with no valid
+// entry the output is zero. Arithmetic as in attend_rows: fp64 scores, exp(s - max), fp64
+// sums, rounded to fp32.
+void attend_list(const Cache& C, int l, int b, int h, int64_t n, const int32_t* list, int k,
+                 const float* const* qs, int G, float scale, float* const* outs) {
+    const int D = C.D;
+    std::vector<int64_t> pos;
+    for (int j = 0; j < k; ++j)
+        if (list[j] >= 0 && list[j] < n) pos.push_back(list[j]);
+    const size_t m = pos.size();
+    if (m == 0) {
+        for (int g = 0; g < G; ++g)
+            for (int c = 0; c < D; ++c) outs[g][c] = 0.0f;
+        return;
+    }
+    std::vector<double> sc((size_t)G * m);
+    std::vector<float> row(D);
+    for (size_t j = 0; j < m; ++j) {
+        position_row(C, l, b, h, 0, pos[j], n, row.data());
+        for (int g = 0; g < G; ++g) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c) acc += (double)qs[g][c] * (double)row[c];
+            sc[(size_t)g * m + j] = (double)scale * acc;
+        }
+    }
+    std::vector<double> mx(G, -INFINITY), den(G, 0.0), o((size_t)G * D, 0.0);
+    for (int g = 0; g < G; ++g)
+        for (size_t j = 0; j < m; ++j) mx[g] = std::max(mx[g], sc[(size_t)g * m + j]);
+    for (size_t j = 0; j < m; ++j) {
+        position_row(C, l, b, h, 1, pos[j], n, row.data());
+        for (int g = 0; g < G; ++g) {
+            double p = std::exp(sc[(size_t)g * m + j] - mx[g]);
+            den[g] += p;
+            for (int c = 0; c < D; ++c) o[(size_t)g * D + c] += p * (double)row[c];
+        }
+    }
+    for (int g = 0; g < G; ++g)
+        for (int c = 0; c < D; ++c) outs[g][c] = (float)(o[(size_t)g * D + c] / den[g]);
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -646,6 +689,30 @@ int orc_decode(void* c, int l, const float* q, float scale, float* out, int nthr
             os[g] = out + off;
         }
         attend_rows(C, l, b, h, n, n, qs.data(), G, scale, os.data());
+    });
+    return OK;
+}
+
+// Index-gather decode: like orc_decode, but each (batch, kv head) attends only to the k
+// positions listed in idx[b][h][0..k) (see attend_list for the reading of the list).
+// q, out: fp32 [B][Hq][D]; idx: int32 [B][H][k].
+int orc_decode_indexed(void* c, int l, const float* q, float scale, const int32_t* idx, int k, float* out,
+                       int nthreads) {
+    Cache& C = *(Cache*)c;
+    if (l < 0 || l >= C.L || k < 1) return ERR_INVALID_ARG;
+    const int64_t n = C.n[l];
+    if (n == 0) return ERR_EMPTY;
+    const int G = C.Hq / C.H;
+    parallel_for((int64_t)C.B * C.H, nthreads, [&](int64_t u) {
+        int b = (int)(u / C.H), h = (int)(u % C.H);
+        std::vector<const float*> qs(G);
+        std::vector<float*> os(G);
+        for (int g = 0; g < G; ++g) {
+            size_t off = ((size_t)b * C.Hq + h * G + g) * C.D;
+            qs[g] = q + off;
+            os[g] = out + off;
+        }
+        attend_list(C, l, b, h, n, idx + (size_t)u * k, k, qs.data(), G, scale, os.data());
     });
     return OK;
 }
