@@ -697,6 +697,40 @@ def supplementary(dev, peaks):
     del c, ks, vs
     torch.cuda.empty_cache()
 
+    # index-gather decode (QSA budget): one full-length layer, 2,048 listed positions per kv
+    # head (the 16 newest, in the ring, and 2,032 seeded others), L2 flushed before each call
+    n = N_FILL + C_PF
+    c = kvq.KVCache(1, 1, H_, HQ_, D_, n, K_FMT, V_FMT, T_FMT, W_, device=dev)
+    fill(c, 1, H_, D_, n)
+    gen.manual_seed(11)
+    k_list = 2048
+    lists = []
+    for h in range(H_):
+        rest = torch.randperm(n - 16, generator=gen, device=dev)[:k_list - 16]
+        lists.append(torch.cat([torch.arange(n - 16, n, device=dev), rest]))
+    idx = torch.stack(lists)[None].to(torch.int32).contiguous()
+    in_ring = (idx >= n - W_)
+    gbytes = int(in_ring.sum()) * 2 * ROW_T + int((~in_ring).sum()) * (ROW_K + ROW_V) + 2 * HQ_ * D_ * 4
+    q = torch.randn(1, HQ_, D_, device=dev, generator=gen) / math.sqrt(D_)
+    out = torch.empty_like(q)
+    ws = c.ensure_workspace(1)
+    ts = []
+    for i in range(13):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvq.kvq_decode_attention_indexed(c.handle, 0, q, 1.0, idx, k_list, out, ws, ws.numel())
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(e0.elapsed_time(e1) / 1e3)
+    tg = statistics.median(ts)
+    res["index_gather_2048"] = {"us": tg * 1e6, "gathered_bytes": gbytes, "gbs": gbytes / tg / 1e9,
+                                "context": n, "positions_per_kv_head": k_list,
+                                "note": "latency-bound: 3.2 MB gathered per call"}
+    del c, idx
+    torch.cuda.empty_cache()
+
     # KVarN: batch 8, 2 kv heads, 131,072 positions
     B, H, Hq, D, n = 8, 2, 16, 256, 131072
     c = kvq.KVCache(1, B, H, Hq, D, n, K_FMT, V_FMT, 14, 0, kvarn=1, device=dev)

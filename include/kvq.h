@@ -157,6 +157,19 @@ KVQ_API kvq_status kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t n_
 KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const float* q, float scale,
                                 float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Index-gather decode ([OFFLOAD], the QSA paragraph: an indexer picks a budget of 2,048
+ * positions per step and attention reads only those rows of the quantized cache): like
+ * kvq_decode_attention, but each (batch element, kv head) attends only to the positions
+ * it lists. idx: device int32 [batch][n_kv_heads][n_idx], 4-byte aligned, 1 <= n_idx <=
+ * KVQ_MAX_GATHER. Entries outside [0, n) are skipped; the others enter the softmax in list
+ * order, a repeated position counting once per entry; a list without a valid entry gives a
+ * zero output. Rows are fetched by one bulk copy each from the low-bit store or the ring,
+ * wherever the position lies. ws: >= kvq_decode_workspace_bytes(cache, 1). */
+#define KVQ_MAX_GATHER 65536
+KVQ_API kvq_status kvq_decode_attention_indexed(kvq_cache* cache, int32_t layer, const float* q, float scale,
+                                        const int32_t* idx, int32_t n_idx, float* out, void* ws,
+                                        size_t ws_bytes, void* stream);
+
 /* Causal chunked-prefill attention for the n_chunk positions just appended ([HARDNUM]
  * "Engine speed and cache reuse": prompt processing with the config D cache; chunk row i
  * sits at position n - n_chunk + i and attends to positions <= its own over the

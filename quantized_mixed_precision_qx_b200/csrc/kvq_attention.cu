@@ -36,6 +36,8 @@ struct P1Args {
     long long region_rows; // rows of this region (n_main or n_ring)
     int split_offset;      // first split index of this region
     int n_split;           // total splits per (b, row, h)
+    const int* idx;        // index-gather decode: [B][H][n_idx] positions, or nullptr
+    int n_idx;
 };
 
 template <int CPL>
@@ -53,7 +55,8 @@ attn_pass1(P1Args a) {
     const long long t0 = (long long)split * a.chunk;
     long long t1 = t0 + a.chunk;
     if (t1 > a.region_rows) t1 = a.region_rows;
-    if (!a.ring && t1 > limit + 1) t1 = limit + 1;   // main rows: index == position
+    if (!a.ring && !a.idx && t1 > limit + 1) t1 = limit + 1;   // main rows: index == position
+    const int* il = a.idx ? a.idx + ((long long)br * H + h) * a.n_idx : nullptr;
 
     const int kvarn = lv.kvarn && !a.ring;
     const float* sK = kvarn ? lv.scales + ((long long)(b * H + h) * 2 + 0) * D : nullptr;
@@ -91,14 +94,26 @@ attn_pass1(P1Args a) {
     }
 
     for (long long t = t0 + warp; t < t1; t += P1_WARPS) {
-        if (a.ring) {
+        long long row = t;
+        if (il) {
+            // gather: list entry t names a position; this pass takes those of its region
+            const long long p = il[t];
+            const long long ring0 = lv.W ? a.n - lv.W : a.n;
+            if (a.ring) {
+                if (p < 0 || p < ring0 || p >= a.n) continue;
+                row = p % lv.W;
+            } else {
+                if (p < 0 || p >= ring0) continue;
+                row = p;
+            }
+        } else if (a.ring) {
             const long long W = lv.W;
             const long long pos = ring_base + ((t - ring_base) % W + W) % W;
             if (pos > limit) continue;
         }
         float kx[CPL], vx[CPL];
-        load_row_values<CPL>(kbase + t * fk.stride, fk, lane, kx);
-        load_row_values<CPL>(vbase + t * fv.stride, fv, lane, vx);
+        load_row_values<CPL>(kbase + row * fk.stride, fk, lane, kx);
+        load_row_values<CPL>(vbase + row * fv.stride, fv, lane, vx);
         float s[MAXG];
 #pragma unroll
         for (int g = 0; g < MAXG; ++g) {
@@ -233,7 +248,8 @@ __global__ void __launch_bounds__(32 * MG) attn_merge(const float* __restrict__ 
             Lt = fmaf(sm_l[j][lane], w, Lt);
             Ot = fmaf(sm_o[j][lane], w, Ot);
         }
-        out[(br * H * G + hq) * (long long)D + c] = Ot / Lt;
+        // no position at all (an index list without a valid entry): zero output
+        out[(br * H * G + hq) * (long long)D + c] = Lt > 0.f ? Ot / Lt : 0.f;
     }
 }
 
@@ -310,8 +326,10 @@ SplitPlan plan_splits(long long n_main, long long n_ring, long long units, int n
 
 cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, float* out,
                              float* ws, long long n, int rows, const SplitPlan& plan,
-                             cudaStream_t st) {
+                             cudaStream_t st, const int* idx, int n_idx) {
     P1Args a{};
+    a.idx = idx;
+    a.n_idx = n_idx;
     a.lv = lv;
     a.q = q;
     a.qscale = scale * LOG2E;
@@ -331,7 +349,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
         const int region = 1 - ri;
         a.ring = region;
         a.chunk = region ? plan.ring_chunk : plan.main_chunk;
-        a.region_rows = region ? n_ring : n_main;
+        a.region_rows = idx ? n_idx : (region ? n_ring : n_main);
         a.split_offset = region ? plan.n_main_split : 0;
         const int ns = region ? plan.n_ring_split : plan.n_main_split;
         if (ns == 0) continue;
@@ -364,6 +382,9 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
             t.H = lv.H;
             t.G = lv.G;
             t.D = lv.D;
+            t.idx = idx;
+            t.n_idx = n_idx;
+            t.ring_start = lv.W ? n - lv.W : n;
             t.dependent = launched ? 1 : 0;
             const dim3 grid(ns, lv.H, lv.B * rows);
             e = tc::launch_tc(fk.id, fv.id, t, grid, tc::smem_bytes(fk.stride, fv.stride, lv.D, tc::query_parts(fk.id)), st);

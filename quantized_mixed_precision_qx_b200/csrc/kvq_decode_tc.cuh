@@ -54,6 +54,11 @@ struct Args {
     long long region_stride_k, region_stride_v;   // bytes between (b, h) regions
     int split_offset, n_split;
     int H, G, D;
+    // index-gather decode: per (batch, kv head) a list of n_idx positions (splits then run
+    // over list entries); entries outside this region's positions are masked out
+    const int* idx;         // [B][H][n_idx] or nullptr
+    int n_idx;
+    long long ring_start;   // first position held in the ring (n - W; n when W == 0)
     // 0: first launch of the call (lets the next launch start early);
     // 1: launched as a programmatic dependent of the previous pass: runs concurrently
     //    with it and, before exiting, waits for it to finish, so a later dependent that
@@ -78,7 +83,7 @@ constexpr size_t QSUM_BYTES = NBMAX * 8 * sizeof(float);
 constexpr size_t QEXP_BYTES = 2 * 8 * sizeof(float);     // per head: 2^-e (query scaling), 2^e (score)
 __host__ __device__ constexpr size_t smem_bytes(int ks, int vs, int D, int parts) {
     return main_bytes(ks, vs, D) + PT_BYTES + XS_BYTES + qs_bytes(parts) + QSUM_BYTES + QEXP_BYTES +
-           2 * STAGES * sizeof(uint64_t) + 16;
+           2 * STAGES * sizeof(uint64_t) + STAGES * sizeof(uint64_t) + 16;
 }
 
 
@@ -120,7 +125,9 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     float* qexp_s = qsum_s + NBMAX * 8;                                                  // [2][8]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + mb + PT_BYTES + XS_BYTES + qs_bytes(KP) + QSUM_BYTES + QEXP_BYTES);
     uint64_t* empty = full + STAGES;
-    int* fault = reinterpret_cast<int*>(empty + STAGES);
+    uint64_t* gmask = empty + STAGES;                 // gather mode: rows of each stage that were fetched
+    int* fault = reinterpret_cast<int*>(gmask + STAGES);
+    const bool gather = a.idx != nullptr;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -133,7 +140,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     long long t0 = (long long)split * a.chunk;
     long long t1 = t0 + a.chunk;
     if (t1 > a.region_rows) t1 = a.region_rows;
-    if (!a.ring && t1 > limit + 1) t1 = limit + 1;
+    if (!a.ring && !gather && t1 > limit + 1) t1 = limit + 1;
     if (t1 < t0) t1 = t0;
     const int n_tiles = (int)((t1 - t0 + TOK - 1) / TOK);
 
@@ -164,8 +171,13 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
             for (int sl = 0; sl < 4; ++sl) qv[m][sl] = (g < G) ? qg[32 * warp + q_channel<KF>(t, m, sl)] : 0.f;
     }
     // Rows past the end of a partial last tile are read (and multiplied by p = 0): zero
-    // them in that tile's stage so they always hold finite values.
-    if (n_tiles > 0) {
+    // them in that tile's stage so they always hold finite values. In gather mode any row of
+    // a tile can be masked out: zero both stages (a masked row then holds zeros or an earlier
+    // tile's fetched row).
+    if (gather) {
+        for (size_t i = (size_t)threadIdx.x * 16; i < STAGES * sb; i += THREADS * 16)
+            *reinterpret_cast<uint4*>(stage0 + i) = make_uint4(0, 0, 0, 0);
+    } else if (n_tiles > 0) {
         const int last_rows = (int)(t1 - t0 - (long long)(n_tiles - 1) * TOK);
         if (last_rows < TOK) {
             uint8_t* st = stage0 + ((n_tiles - 1) % STAGES) * sb;
@@ -186,7 +198,67 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
     __syncthreads();
 
     // ------------------------------------------------------------ producer warp
-    if (warp == CWARPS) {
+    if (warp == CWARPS && gather) {
+        // one bulk copy per listed row of this region, issued by the lane that owns the row
+        // (rows lane and lane + 32 of the tile); lane 0 publishes the tile's row mask
+        const int* il = a.idx + ((long long)br * H + h) * a.n_idx;
+        const long long W = a.W;
+        int issued = 0;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int s = it % STAGES;
+            int ok = 1;
+            if (it >= STAGES && lane == 0) ok = mbar_wait(&empty[s], ((it / STAGES) - 1) & 1) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                if (lane == 0) *fault = 1;
+                break;
+            }
+            const long long r0 = t0 + (long long)it * TOK;
+            const int nrows = (int)min((long long)TOK, t1 - r0);
+            long long row[2];
+            bool v[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int rr = lane + 32 * k;
+                v[k] = false;
+                row[k] = 0;
+                if (rr < nrows) {
+                    const long long p = il[r0 + rr];
+                    if (a.ring) {
+                        v[k] = p >= 0 && p >= a.ring_start && p < a.n;
+                        row[k] = v[k] ? p % W : 0;
+                    } else {
+                        v[k] = p >= 0 && p < a.ring_start;
+                        row[k] = p;
+                    }
+                }
+            }
+            const uint32_t m0 = __ballot_sync(0xffffffffu, v[0]), m1 = __ballot_sync(0xffffffffu, v[1]);
+            uint8_t* st = stage0 + s * sb;
+            if (lane == 0) {
+                gmask[s] = (uint64_t)m0 | ((uint64_t)m1 << 32);
+                const uint32_t nv = (uint32_t)(__popc(m0) + __popc(m1));
+                mbar_arrive_expect_tx(&full[s], nv * (uint32_t)(a.kstride + a.vstride));
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                if (v[k]) {
+                    const int rr = lane + 32 * k;
+                    bulk_g2s(st + (size_t)rr * a.kstride, kreg + row[k] * a.kstride, (uint32_t)a.kstride, &full[s]);
+                    bulk_g2s(st + (size_t)TOK * a.kstride + (size_t)rr * a.vstride, vreg + row[k] * a.vstride,
+                             (uint32_t)a.vstride, &full[s]);
+                }
+            }
+            issued = it + 1;
+        }
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % STAGES + STAGES) % STAGES;
+                if (issued > s && last >= 0) mbar_wait(&full[s], (last / STAGES) & 1, 50000000ull);
+            }
+        }
+    } else if (warp == CWARPS) {
         if (lane == 0) {
             int issued = 0;
             for (int it = 0; it < n_tiles; ++it) {
@@ -305,7 +377,9 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
             if (sub0 < nrows) {                      // uniform over the pair
                 const uint8_t* kt = stage0 + s * sb;
                 const uint8_t* vt = kt + (size_t)TOK * a.kstride;
+                const uint64_t gm = gather ? gmask[s] : 0ull;
                 auto valid = [&](int rr) -> bool {
+                    if (gather) return (gm >> (sub0 + rr)) & 1ull;
                     if (sub0 + rr >= nrows) return false;
                     if (a.ring) {
                         long long d = r0 + sub0 + rr + W - nmodw;

@@ -299,6 +299,29 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const float* q, flo
     return attention_common(c, layer, q, 1, scale, out, ws, ws_bytes, stream);
 }
 
+kvq_status kvq_decode_attention_indexed(kvq_cache* c, int32_t layer, const float* q, float scale,
+                                        const int32_t* idx, int32_t n_idx, float* out, void* ws, size_t ws_bytes,
+                                        void* stream) {
+    if (!c || layer < 0 || layer >= c->L.n_layers || !q || !out || !ws || !idx) return KVQ_ERR_INVALID_ARG;
+    if (n_idx < 1 || n_idx > KVQ_MAX_GATHER) return KVQ_ERR_INVALID_ARG;
+    if (!c->buf) return KVQ_ERR_NOT_BOUND;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(ws) || ((uintptr_t)idx & 3)) return KVQ_ERR_ALIGNMENT;
+    const long long n = c->n[layer];
+    if (n == 0) return KVQ_ERR_EMPTY;
+    size_t need = 0;
+    kvq_status s = kvq_decode_workspace_bytes(c, 1, &need);
+    if (s != KVQ_OK) return s;
+    if (ws_bytes < need) return KVQ_ERR_CAPACITY;
+    const LayerView lv = layer_view(c, layer);
+    // both passes walk the whole list; a pass whose region holds no position is skipped
+    const long long list_main = (c->W == 0 || n > c->W) ? n_idx : 0;
+    const long long list_ring = c->W ? n_idx : 0;
+    const long long units = (long long)c->L.batch * c->L.n_kv_heads;
+    const int tc_ctas = use_tensor_cores(c->L.head_dim) ? tc_ctas_per_sm(c->L.head_dim) : 0;
+    const SplitPlan plan = plan_splits(list_main, list_ring, units, c->num_sms, tc_ctas);
+    return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, 1, plan, (cudaStream_t)stream, idx, n_idx));
+}
+
 kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, int32_t n_chunk, float scale,
                                  float* out, void* ws, size_t ws_bytes, void* stream) {
     if (n_chunk < 1) return KVQ_ERR_INVALID_ARG;

@@ -141,9 +141,11 @@ size_t partial_floats(int G, int D);   // floats of one split partial
 // rows = query rows per (b, h): 1 for decode, n_chunk for prefill. q/out layout
 // [B][rows][Hq][D]. pos_base: position of query row 0 (n - rows); decode uses rows = 1
 // and pos_base = n - 1 so every row sees all n positions.
+// idx (optional): index-gather decode (rows = 1), [B][H][n_idx] positions per (b, h); the
+// low-bit and ring passes then both run over the list entries.
 cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, float* out,
                              float* ws, long long n, int rows, const SplitPlan& plan,
-                             cudaStream_t st);
+                             cudaStream_t st, const int* idx = nullptr, int n_idx = 0);
 
 // Chunked prefill on tcgen05 (head_dim 128 / 256): q, out [B][C][Hq][D], n = cached
 // positions after the chunk's append.

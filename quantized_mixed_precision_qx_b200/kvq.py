@@ -27,7 +27,8 @@ EXPORTED = ["kvq_cache_create", "kvq_cache_required_bytes", "kvq_cache_bind", "k
             "kvq_append", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_prefill_attention",
             "kvq_length", "kvq_set_channel_scales", "kvq_export_blocks", "kvq_status_string",
             "kvq_decode_attention_noalloc", "kvq_get_channel_scales", "kvq_device_status",
-            "kvq_selftest_wait_timeout"]
+            "kvq_selftest_wait_timeout", "kvq_decode_attention_indexed"]
+MAX_GATHER = 65536                    # KVQ_MAX_GATHER
 NOALLOC_WORKSPACE_BYTES = 8 << 20     # KVQ_NOALLOC_WORKSPACE_MIB
 
 
@@ -65,6 +66,7 @@ def lib():
             "kvq_decode_attention": [p, i32, p, f32, p, p, sz, p],
             "kvq_prefill_attention": [p, i32, p, i32, f32, p, p, sz, p],
             "kvq_decode_attention_noalloc": [p, i32, p, f32, p, p],
+            "kvq_decode_attention_indexed": [p, i32, p, f32, p, i32, p, p, sz, p],
             "kvq_length": [p, i32, ctypes.POINTER(i64)],
             "kvq_set_channel_scales": [p, i32, p, p, p],
             "kvq_get_channel_scales": [p, i32, p, p],
@@ -137,6 +139,12 @@ def kvq_decode_workspace_bytes(cache, n_query_rows: int) -> int:
 def kvq_decode_attention(cache, layer: int, q, scale: float, out, ws, ws_bytes: int, stream=None):
     _check(lib().kvq_decode_attention(cache, layer, _dptr(q), scale, _dptr(out), _dptr(ws), ws_bytes,
                                       _stream(stream)), "kvq_decode_attention")
+
+
+def kvq_decode_attention_indexed(cache, layer: int, q, scale: float, idx, n_idx: int, out, ws, ws_bytes: int,
+                                 stream=None):
+    _check(lib().kvq_decode_attention_indexed(cache, layer, _dptr(q), scale, _dptr(idx), n_idx, _dptr(out),
+                                              _dptr(ws), ws_bytes, _stream(stream)), "kvq_decode_attention_indexed")
 
 
 def kvq_prefill_attention(cache, layer: int, q, n_chunk: int, scale: float, out, ws, ws_bytes: int, stream=None):
@@ -229,6 +237,15 @@ class KVCache:
             out = torch.empty_like(q)
         ws = self.ensure_workspace(1)
         kvq_decode_attention(self.handle, layer, q, scale, out, ws, ws.numel(), stream)
+        return out
+
+    def decode_indexed(self, layer, q, idx, scale=1.0, out=None, stream=None):
+        """idx: int32 device tensor [batch][n_kv_heads][n_idx]."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        ws = self.ensure_workspace(1)
+        kvq_decode_attention_indexed(self.handle, layer, q, scale, idx, idx.shape[2], out, ws, ws.numel(), stream)
         return out
 
     def prefill(self, layer, q, scale=1.0, out=None, stream=None):

@@ -7,7 +7,8 @@ benchmark uses, on outputs the oracle computes one by one:
 - KVarN at batch 8 x 2 KV heads x 131,072;
 - the full-length cache on two seeded layers: fill 257,984, append the 4,096-row chunk,
   prefill it (rows on both sides of the window boundary and seeded random rows), then 8 of
-  its (append 1 + decode) steps at 262,081..262,088.
+  its (append 1 + decode) steps at 262,081..262,088, and an index-gather decode of 2,048
+  positions per kv head.
 Stored bytes of sampled position ranges and the whole ring are bit-exact; decode and
 prefill outputs are within the stated tolerance.
 
@@ -118,6 +119,16 @@ def test_full_length_two_layers():
             check_close(g.decode(layer, to_dev(qd), 1.0).cpu().numpy(), o.decode(layer, qd, 1.0), vmax,
                         f"full-length decode layer {layer} step {s} n={n + s + 1}")
         _bytes_sampled(g, o, B, H, n + steps, W, [(n - W - 8, 16)], layer)
+        # index-gather decode with the QSA budget: 2,048 seeded positions per kv head over the
+        # whole context, the newest ones (in the ring) included
+        import torch
+        rng = np.random.default_rng(50 + layer)
+        nn = n + steps
+        idx = np.stack([np.concatenate([np.arange(nn - 16, nn), rng.choice(nn - 16, 2032, replace=False)])
+                        for _ in range(H)])[None].astype(np.int32)
+        qd = wl.q_decode(layer, 100)
+        out = g.decode_indexed(layer, to_dev(qd), torch.from_numpy(idx).cuda(), 1.0).cpu().numpy()
+        check_close(out, o.decode_indexed(layer, qd, idx, 1.0), vmax, f"full-length gather layer {layer}")
 
 
 def test_kvarn_full():
