@@ -57,7 +57,7 @@ def lib():
             "orc_unpack_block": (c_i, [c_i, c_p, c_p, c_p, c_p]),
             "orc_quantize_row": (c_i, [c_i, c_p, c_i, c_p]),
             "orc_dequant_row": (c_i, [c_i, c_p, c_i, c_p]),
-            "orc_cache_new": (c_p, [c_i, c_i, c_i, c_i, c_i, c_i64, c_i, c_i, c_i, c_i, c_i, c_i, c_d]),
+            "orc_cache_new": (c_p, [c_i, c_i, c_i, c_i, c_i, c_i64, c_i, c_i, c_i, c_i, c_i, c_i, c_d, c_i]),
             "orc_cache_free": (None, [c_p]),
             "orc_length": (c_i64, [c_p, c_i]),
             "orc_set_channel_scales": (c_i, [c_p, c_i, c_p, c_p]),
@@ -168,12 +168,13 @@ class Cache:
     """Oracle cache: same semantics as the library's cache, canonical bytes."""
 
     def __init__(self, n_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx,
-                 k_fmt, v_fmt, tail_fmt=NONE, W=0, kvarn=0, calib=512, eps=1e-6, threads=None):
+                 k_fmt, v_fmt, tail_fmt=NONE, W=0, kvarn=0, calib=512, eps=1e-6, threads=None, kivi=0):
         self.L, self.B, self.H, self.Hq, self.D = n_layers, batch, n_kv_heads, n_q_heads, head_dim
         self.max_ctx, self.kf, self.vf, self.tf, self.W = max_ctx, k_fmt, v_fmt, tail_fmt, W
+        self.kivi = kivi
         self.threads = threads or (os.cpu_count() or 1)
         self._h = lib().orc_cache_new(n_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx,
-                                      k_fmt, v_fmt, tail_fmt, W, kvarn, calib, eps)
+                                      k_fmt, v_fmt, tail_fmt, W, kvarn, calib, eps, kivi)
         if not self._h:
             raise ValueError("oracle rejected the cache description")
 
@@ -207,8 +208,15 @@ class Cache:
         return sK, sV
 
     def export(self, layer, b, h, kv, region, pos0, count):
+        """region 0: low-bit rows pos0.. (per-channel K: groups pos0.., D blocks each);
+        region 1: ring slots; region 2 (per-channel K): pending slots as fp32 rows."""
         f = (self.tf if region == 1 else (self.vf if kv else self.kf))
-        out = np.empty(count * row_bytes(f, self.D), dtype=np.uint8)
+        if region == 2:
+            out = np.empty(count * self.D * 4, dtype=np.uint8)
+        elif region == 0 and kv == 0 and self.kivi:
+            out = np.empty(count * self.D * block_bytes(self.kf), dtype=np.uint8)
+        else:
+            out = np.empty(count * row_bytes(f, self.D), dtype=np.uint8)
         self._chk(lib().orc_export(self._h, layer, b, h, kv, region, pos0, count, _ptr(out)), "export")
         return out
 

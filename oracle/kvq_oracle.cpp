@@ -333,20 +333,35 @@ void dequant_row(int f, const uint8_t* in, int D, float* x) {
 // KVarN ([BEELLAMA] names it; READING fixed by the workload definition):
 //  s_c = fp32(sqrt(S/T + eps)), S = sum over the first T tokens of x^2 in fp64 with a
 //  fixed pairwise tree; blocks quantize x / s_c; dequant multiplies by s_c.
+// Per-channel K ([HARDNUM] "Reddit reactions": quantizing K along the token axis, as
+// KIVI does, instead of 32 values per token; READING of its details):
+//  * a K block is 32 consecutive positions of one channel: group g of channel c holds
+//    the values of positions 32g .. 32g + 31, quantized with the same qX_0 / qX_1 rule;
+//  * the value of a position entering the K store is the same as for per-token blocks
+//    (deq_tail(Q_tail(x)) with a ring, x without one);
+//  * a group is quantized when its last position enters the K store (leaves the window);
+//    until then the positions that have entered are held exactly (fp32) in a 32-row
+//    pending buffer, slot pos mod 32, and attention reads them from there;
+//  * V keeps per-token blocks; per-channel K is not combined with KVarN.
 // ---------------------------------------------------------------------------
 struct Cache {
     int L, B, H, Hq, D;
     int64_t max_ctx;
     int kf, vf, tf, W;
     int kvarn, calib;
+    int kivi;                                     // per-channel (token-axis) K blocks
     double eps;
     std::vector<int64_t> n;                       // per layer
     std::vector<std::vector<uint8_t>> main_;      // [L][B][H][2] rows of max_ctx
     std::vector<std::vector<uint8_t>> ring;       // [L][B][H][2] rows of W
     std::vector<float> s;                         // [L][B][H][2][D]
     std::vector<char> s_set;                      // [L]
+    std::vector<std::vector<float>> pend;         // per-channel K: [L][B][H] 32 x D pending values
 
     size_t unit(int l, int b, int h, int kv) const { return (((size_t)l * B + b) * H + h) * 2 + kv; }
+    size_t head(int l, int b, int h) const { return ((size_t)l * B + b) * H + h; }
+    // per-channel K: block of channel c of group g, canonical bytes
+    size_t group_block(int64_t g, int c) const { return ((size_t)g * D + c) * block_bytes(kf); }
     int low_fmt(int kv) const { return kv ? vf : kf; }
     size_t row_bytes(int f) const { return (size_t)block_bytes(f) * (D / 32); }
 };
@@ -369,10 +384,30 @@ void kvarn_divide(const float* x, const float* s, int D, float* y) {
     for (int c = 0; c < D; ++c) y[c] = x[c] / s[c];
 }
 
+// Per-channel K: position pos enters the K store with values x (one per channel): it is
+// held in pending slot pos mod 32; the last position of a group completes it, and every
+// channel's 32 values are quantized into that channel's block of the group.
+void store_kivi(Cache& C, int l, int b, int h, int64_t pos, const float* x) {
+    const int D = C.D;
+    float* pend = C.pend[C.head(l, b, h)].data();
+    std::memcpy(pend + (size_t)(pos % 32) * D, x, sizeof(float) * D);
+    if (pos % 32 != 31) return;
+    const int64_t g = pos / 32;
+    float vals[32];
+    uint8_t codes[32];
+    for (int c = 0; c < D; ++c) {
+        for (int t = 0; t < 32; ++t) vals[t] = pend[(size_t)t * D + c];
+        uint16_t d16 = 0, m16 = 0;
+        quantize_codes(C.kf, vals, 32, codes, &d16, &m16);
+        pack_block(C.kf, codes, d16, m16, &C.main_[C.unit(l, b, h, 0)][C.group_block(g, c)]);
+    }
+}
+
 // Quantize one raw row x into the low-bit main store slot `pos`, via the tail
 // format when the cache has a ring (the row then passed through the ring).
 void store_low(Cache& C, int l, int b, int h, int kv, int64_t pos, const float* x_raw) {
     const int D = C.D;
+    if (kv == 0 && C.kivi) { store_kivi(C, l, b, h, pos, x_raw); return; }
     const int f = C.low_fmt(kv);
     std::vector<float> y(x_raw, x_raw + D);
     if (C.kvarn) kvarn_divide(x_raw, &C.s[C.unit(l, b, h, kv) * D], D, y.data());
@@ -420,6 +455,22 @@ void position_row(const Cache& C, int l, int b, int h, int kv, int64_t pos, int6
     const size_t u = C.unit(l, b, h, kv);
     if (C.W > 0 && pos >= n - C.W) {
         dequant_row(C.tf, &C.ring[u][(size_t)(pos % C.W) * C.row_bytes(C.tf)], D, out);
+        return;
+    }
+    if (kv == 0 && C.kivi) {
+        // positions below the window: in a completed group, or still pending
+        const int64_t in_store = C.W > 0 ? std::max<int64_t>(0, n - C.W) : n;
+        if (pos >= in_store / 32 * 32) {
+            const float* pend = C.pend[C.head(l, b, h)].data();
+            std::memcpy(out, pend + (size_t)(pos % 32) * D, sizeof(float) * D);
+            return;
+        }
+        uint8_t codes[32];
+        for (int c = 0; c < D; ++c) {
+            uint16_t d16 = 0, m16 = 0;
+            unpack_block(C.kf, &C.main_[u][C.group_block(pos / 32, c)], codes, &d16, &m16);
+            out[c] = dequant_code(C.kf, d16, m16, codes[pos % 32]);
+        }
         return;
     }
     const int f = C.low_fmt(kv);
@@ -562,8 +613,9 @@ int orc_dequant_row(int f, const uint8_t* in, int D, float* out) {
 }
 
 void* orc_cache_new(int L, int B, int H, int Hq, int D, int64_t max_ctx, int kf, int vf, int tf,
-                    int W, int kvarn, int calib, double eps) {
+                    int W, int kvarn, int calib, double eps, int kivi) {
     if (L < 1 || B < 1 || H < 1 || Hq < H || Hq % H || D < 32 || D % 32 || max_ctx < 1) return nullptr;
+    if (kivi && kvarn) return nullptr;
     if (!is_lowbit(kf) || !is_lowbit(vf)) return nullptr;
     if ((W == 0) != (tf == NONE)) return nullptr;
     if (W < 0 || (W > 0 && !is_tail(tf))) return nullptr;
@@ -571,7 +623,7 @@ void* orc_cache_new(int L, int B, int H, int Hq, int D, int64_t max_ctx, int kf,
     Cache* C = new Cache();
     C->L = L; C->B = B; C->H = H; C->Hq = Hq; C->D = D; C->max_ctx = max_ctx;
     C->kf = kf; C->vf = vf; C->tf = tf; C->W = W;
-    C->kvarn = kvarn; C->calib = calib; C->eps = eps;
+    C->kvarn = kvarn; C->calib = calib; C->eps = eps; C->kivi = kivi ? 1 : 0;
     C->n.assign(L, 0);
     const size_t units = (size_t)L * B * H * 2;
     C->main_.resize(units);
@@ -582,9 +634,12 @@ void* orc_cache_new(int L, int B, int H, int Hq, int D, int64_t max_ctx, int kf,
                 for (int kv = 0; kv < 2; ++kv) {
                     size_t u = C->unit(l, b, h, kv);
                     C->main_[u].assign((size_t)max_ctx * C->row_bytes(C->low_fmt(kv)), 0);
+                    if (kv == 0 && C->kivi)   // whole groups of 32 positions
+                        C->main_[u].assign((size_t)((max_ctx + 31) / 32) * C->group_block(1, 0), 0);
                     if (W > 0) C->ring[u].assign((size_t)W * C->row_bytes(tf), 0);
                 }
     C->s.assign(units * D, 1.0f);
+    if (C->kivi) C->pend.assign(units / 2, std::vector<float>((size_t)32 * D, 0.0f));
     C->s_set.assign(L, 0);
     return C;
 }
@@ -648,6 +703,18 @@ int orc_export(void* c, int l, int b, int h, int kv, int region, int64_t pos0, i
     Cache& C = *(Cache*)c;
     if (l < 0 || l >= C.L || b < 0 || b >= C.B || h < 0 || h >= C.H || kv < 0 || kv > 1) return ERR_INVALID_ARG;
     const size_t u = C.unit(l, b, h, kv);
+    if (region == 0 && kv == 0 && C.kivi) {
+        // per-channel K: groups pos0 .. pos0 + count - 1, each its D channel blocks in order
+        if (pos0 < 0 || count < 0 || pos0 + count > (C.max_ctx + 31) / 32) return ERR_INVALID_ARG;
+        std::memcpy(dst, &C.main_[u][C.group_block(pos0, 0)], (size_t)count * C.group_block(1, 0));
+        return OK;
+    }
+    if (region == 2) {
+        // per-channel K pending slots pos0 .. pos0 + count - 1 as fp32 rows of D values
+        if (!C.kivi || kv != 0 || pos0 < 0 || count < 0 || pos0 + count > 32) return ERR_INVALID_ARG;
+        std::memcpy(dst, &C.pend[C.head(l, b, h)][(size_t)pos0 * C.D], (size_t)count * C.D * sizeof(float));
+        return OK;
+    }
     if (region == 0) {
         if (pos0 < 0 || count < 0 || pos0 + count > C.max_ctx) return ERR_INVALID_ARG;
         size_t rb = C.row_bytes(C.low_fmt(kv));
