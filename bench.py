@@ -756,6 +756,19 @@ def supplementary(dev, peaks):
         del c
         torch.cuda.empty_cache()
     res["asymmetric_sweep"] = sweep
+
+    # per-channel K decode (CUDA-core path): 4 kv heads x 256, 65,536 positions, K q5_0 per
+    # channel, V q5_0, no tail
+    B, H, Hq, D, n = 1, 4, 24, 256, 65536
+    c = kvq.KVCache(1, B, H, Hq, D, n, 6, 6, 14, 0, device=dev, k_per_channel=1)
+    t_fill = fill(c, B, H, D, n)
+    td = time_decode(c, B, Hq, D)
+    dbytes = B * H * n * 2 * rows_bytes(6, D) + 2 * B * Hq * D * 4
+    res["per_channel_k"] = {"decode_gbs": dbytes / td / 1e9, "decode_frac": dbytes / td / 1e9 / peak,
+                            "decode_us": td * 1e6, "append_fill_mtok_s": n * B / t_fill / 1e6,
+                            "note": "K q5_0 per channel (token-axis blocks), V q5_0, no tail; CUDA-core attention"}
+    del c
+    torch.cuda.empty_cache()
     res["quality_rel_l2_vs_fp32"] = quality(dev)
     return res
 
@@ -786,13 +799,19 @@ def quality(dev):
     vv = v.double().permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
     refs = [torch.softmax(torch.einsum("bhd,bhnd->bhn", q.double(), kk), dim=-1).unsqueeze(2).matmul(vv).squeeze(2)
             for q in qs]
-    cases = [(name, f, f, kvq.NONE, 0) for f, name in enumerate(FMT_NAMES)]
-    cases += [(f"K-only {name}", f, kvq.Q8_1, kvq.NONE, 0) for f, name in enumerate(FMT_NAMES)]
-    cases += [(f"V-only {name}", kvq.Q8_1, f, kvq.NONE, 0) for f, name in enumerate(FMT_NAMES)]
-    cases.append(("q6_0/q5_0 + q8_0 tail 2048", K_FMT, V_FMT, T_FMT, W_))
+    cases = [(name, f, f, kvq.NONE, 0, 0) for f, name in enumerate(FMT_NAMES)]
+    cases += [(f"K-only {name}", f, kvq.Q8_1, kvq.NONE, 0, 0) for f, name in enumerate(FMT_NAMES)]
+    cases += [(f"V-only {name}", kvq.Q8_1, f, kvq.NONE, 0, 0) for f, name in enumerate(FMT_NAMES)]
+    cases.append(("q6_0/q5_0 + q8_0 tail 2048", K_FMT, V_FMT, T_FMT, W_, 0))
+    # per-channel (token-axis) K against per-token K, V q8_1, without and with a 2,048 q8_0 tail
+    for f in (kvq.Q4_0, kvq.Q5_0, kvq.Q6_0):
+        for tf, W in ((kvq.NONE, 0), (kvq.Q8_0, W_)):
+            tail = "no tail" if W == 0 else "q8_0 tail 2048"
+            cases.append((f"K-only {FMT_NAMES[f]} per-token, {tail}", f, kvq.Q8_1, tf, W, 0))
+            cases.append((f"K-only {FMT_NAMES[f]} per-channel, {tail}", f, kvq.Q8_1, tf, W, 1))
     res = {}
-    for name, kf, vf, tf, W in cases:
-        c = kvq.KVCache(1, B, H, Hq, D, n, kf, vf, tf, W, device=dev)
+    for name, kf, vf, tf, W, kpc in cases:
+        c = kvq.KVCache(1, B, H, Hq, D, n, kf, vf, tf, W, device=dev, k_per_channel=kpc)
         for t in range(0, n, 4096):
             c.append(0, k[:, t:t + 4096].contiguous(), v[:, t:t + 4096].contiguous())
         ws = c.ensure_workspace(1)

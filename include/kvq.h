@@ -79,7 +79,13 @@ typedef enum kvq_fmt {
  * blocks ([BEELLAMA] names KVarN): per (layer, batch, kv head, channel, K|V)
  * s = fp32(sqrt(S / T + eps)), S the fp64 sum of x^2 over the first T =
  * kvarn_calib_tokens tokens (a power of two, 64..1024) taken as a fixed pairwise tree;
- * blocks store x / s and are read back as s * value. */
+ * blocks store x / s and are read back as s * value.
+ * k_per_channel = 1 quantizes K along the token axis ([HARDNUM] "Reddit reactions": the KIVI
+ * question; per-channel K reduced the error without a window and did not beat per-token blocks
+ * with the 2k window): a K block holds 32 consecutive positions of one channel, quantized with
+ * the same rules when the last of them enters the K store; positions that entered before
+ * their group is complete are kept exactly (float32) until it is. V keeps per-token blocks.
+ * Not combined with kvarn. Attention over such a cache runs on the CUDA-core path. */
 typedef struct kvq_layout {
     int32_t n_layers;
     int32_t batch;
@@ -89,7 +95,8 @@ typedef struct kvq_layout {
     int32_t kvarn;               /* 0 or 1 */
     int64_t max_ctx;             /* positions per (layer, batch element) */
     int32_t kvarn_calib_tokens;  /* 512 by convention */
-    int32_t reserved;            /* must be 0 */
+    int32_t k_per_channel;       /* 0: K blocks of 32 channels of a token; 1: K blocks of 32
+                                    positions of a channel (see below) */
     double kvarn_eps;            /* 1e-6 by convention */
 } kvq_layout;
 
@@ -140,7 +147,10 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const float* k, c
                       int32_t n_new, void* stream);
 
 /* Workspace bytes for kvq_decode_attention (n_query_rows = 1) or kvq_prefill_attention
- * (n_query_rows = n_chunk). The workspace holds the per-split softmax partials of the
+ * (n_query_rows = n_chunk). For a prefill at head dim 128 / 256 with n_chunk * G > 128 (more
+ * than one 128-row tile of query rows per kv head) the workspace holds the K~ / V~ operand
+ * tiles dequantized once per (batch, kv head): 128 * head_dim bytes per position of max_ctx
+ * per (batch, kv head). Otherwise it holds the per-split softmax partials of the
  * split-K decode ([OFFLOAD]: decode streams the whole attention state each step, so the
  * positions are split across the GPU and the partials merged). KVQ_ERR_NOT_BOUND before a
  * bind (the split count depends on the device's SM count). */
@@ -233,7 +243,10 @@ KVQ_API kvq_status kvq_device_status(kvq_cache* cache, void* stream);
 KVQ_API kvq_status kvq_selftest_wait_timeout(kvq_cache* cache, uint64_t limit_ns, void* stream);
 
 /* Copy stored rows to host memory in the canonical serialisation of [KVBENCH] /
- * [BEELLAMA] block byte counts (per 32-value block:
+ * [BEELLAMA] block byte counts. With k_per_channel, K region 0 copies groups pos0 ..
+ * pos0 + count - 1 (each D canonical blocks in channel order) and K region 2 copies pending
+ * slots pos0 .. (float32 rows of head_dim values, pos0 + count <= 32). Otherwise (per 32-value
+ * block:
  * fp16 d | [fp16 m] | code planes low bits first, little endian; BF16/F16: 32 x 2 bytes).
  * region 0: low-bit store rows pos0..pos0+count-1; region 1: ring slots pos0..+count-1
  * (tail format). kv: 0 = K, 1 = V. Synchronises the device. host_dst must hold

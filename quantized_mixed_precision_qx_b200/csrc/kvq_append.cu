@@ -23,6 +23,8 @@
 // within the append go to the low-bit store directly, through the tail rounding.
 #include "kvq_rowio.cuh"
 
+#include <algorithm>
+
 namespace kvq {
 namespace {
 
@@ -99,8 +101,9 @@ __device__ __forceinline__ void pack_store(uint8_t* p0, uint8_t* p1, int lane, c
         v0 |= (uint64_t)(u[j] & ((1u << W0) - 1)) << (j * W0);
         if constexpr (W1 > 0) v1 |= (uint64_t)(u[j] >> W0) << (j * W1);
     }
-    store_plane_bits(p0, lane, CPL * W0, v0);
-    if constexpr (W1 > 0) store_plane_bits(p1, lane, CPL * W1, v1);
+    // a row of D = 32 * CPL channels has CPL blocks
+    store_plane_bits<CPL>(p0, CPL, lane, W0, v0);
+    if constexpr (W1 > 0) store_plane_bits<CPL>(p1, CPL, lane, W1, v1);
 }
 
 // Quantize this lane's CPL values into row `row` of format f (all lanes participate).
@@ -226,9 +229,53 @@ __device__ __forceinline__ void publish_bounds(uint32_t* st, Bounds bd) {
     }
 }
 
+// The values a ring round trip gives this lane's CPL values (the tail format's rounding,
+// computed in registers; all lanes of the warp participate).
+template <int CPL>
+__device__ __forceinline__ void tail_round(const RowFmt& tail, const float (&x)[CPL], float (&t)[CPL]) {
+    if (tail.kind == 1) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) t[j] = __bfloat162float(__float2bfloat16_rn(x[j]));
+    } else if (tail.kind == 2) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) t[j] = __half2float(__float2half_rn(x[j]));
+    } else {
+        // q8_0 tail: symmetric 8-bit block quantization then exact dequantization
+        constexpr int LPB = Lanes<CPL>::LPB;
+        float a = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
+        a = group_max<LPB>(a);
+        const float d32 = div_range(a, 7);               // a / 127
+        const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
+        float c[CPL];
+        round_codes<CPL, false>(x, d, 0.f, -127.f, 127.f, c);
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) t[j] = __fmul_rn(d, __fsub_rn(c[j], MAGIC));
+    }
+}
+
+// Per-channel K: a position whose group is not complete after this append enters the
+// pending buffer (this lane's CPL values of its float32 row, slot pos mod 32); positions of
+// groups completed by this append were quantized by kivi_group_kernel before this kernel.
+template <int CPL>
+__device__ __forceinline__ void kivi_enter(const LayerView& lv, uint32_t unit, long long pos, uint32_t done, int lane,
+                                           const float (&x)[CPL]) {
+    if (pos < (long long)done) return;
+    float* dst = lv.pend + ((long long)unit * 32 + pos % 32) * lv.D + lane * CPL;
+    if constexpr (CPL % 4 == 0) {
+#pragma unroll
+        for (int j = 0; j < CPL; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) dst[j] = x[j];
+    }
+}
+
 template <int CPL>
 __global__ void __launch_bounds__(32 * WARPS_PER_CTA)
-append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C) {
+append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C,
+              uint32_t kivi_done) {
     const int lane = threadIdx.x & 31;
     // item order: (b, i, h, kv) so consecutive warps read consecutive input rows; the host
     // keeps C * B * H * 2 below 2^32 and positions below 2^31
@@ -248,11 +295,14 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     const uint32_t p = n + i;
 
     uint32_t* st = lv.stats + ((long long)(b * lv.H + h) * 2 + kv) * 2;
+    const bool kivi = lv.kivi && kv == 0;            // per-channel K
+    const uint32_t unit = b * lv.H + h;
     Bounds bd;
     float x[CPL];
     load_row_f32<CPL>(src, lane, x);
 
     if (lv.W == 0) {
+        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, x); return; }
         store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, x, bd);
         publish_bounds(st, bd);
         return;
@@ -261,27 +311,8 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     if (i + W < C) {
         // enters and leaves the window inside this append: tail rounding, then low-bit
         float t[CPL];
-        // round through the tail format in registers (same values a ring round trip gives)
-        if (lv.tail.kind == 1) {
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) t[j] = __bfloat162float(__float2bfloat16_rn(x[j]));
-        } else if (lv.tail.kind == 2) {
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) t[j] = __half2float(__float2half_rn(x[j]));
-        } else {
-            // q8_0 tail: symmetric 8-bit block quantization then exact dequantization
-            constexpr int LPB = Lanes<CPL>::LPB;
-            float a = 0.f;
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) a = fmaxf(a, fabsf(x[j]));
-            a = group_max<LPB>(a);
-            const float d32 = div_range(a, 7);               // a / 127
-            const float d = __half2float(__float2half_rn(fminf(d32, 65504.f)));
-            float c[CPL];
-            round_codes<CPL, false>(x, d, 0.f, -127.f, 127.f, c);
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) t[j] = __fmul_rn(d, __fsub_rn(c[j], MAGIC));
-        }
+        tail_round<CPL>(lv.tail, x, t);
+        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, t); return; }
         store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, t, bd);
         publish_bounds(st, bd);
         return;
@@ -297,12 +328,113 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
         float y[CPL];
         load_row_values<CPL>(srow, lv.tail, lane, y);
         __syncwarp();
-        store_low<CPL>(main + (long long)q * fl.stride, fl, s, lane, y, bd);
+        if (kivi) kivi_enter<CPL>(lv, unit, q, kivi_done, lane, y);
+        else store_low<CPL>(main + (long long)q * fl.stride, fl, s, lane, y, bd);
     }
     __syncwarp();
     const float rb = store_row<CPL>(srow, lv.tail, lane, x);   // ring rows hold raw values
     bd.add(rb, rb);
     publish_bounds(st, bd);
+}
+
+// Per-channel K, groups completed by an append of C positions to a cache of n0: one CTA per
+// (batch, kv head, group). Its 8 warps gather the group's 32 rows as they enter the K store
+// (pending rows for positions that entered earlier, ring rows for positions leaving the
+// window now, tail-rounded input rows for positions that enter and leave in this append,
+// raw input rows without a ring) into shared memory; then thread c quantizes channel c's
+// 32 values into its canonical block (same rules as a per-token block: absmax or min/max,
+// division-free exact scale, rhaz codes) and writes it. Runs before append_kernel, which
+// overwrites the ring slots and the pending rows.
+template <int CPL>
+__global__ void __launch_bounds__(256)
+kivi_group_kernel(LayerView lv, const float* __restrict__ k, uint32_t n0, uint32_t C, uint32_t g0, uint32_t ngroups) {
+    extern __shared__ float sg[];                        // [32][D]
+    const int D = lv.D;
+    const uint32_t unit = blockIdx.x / ngroups;          // b * H + h
+    const uint32_t g = g0 + blockIdx.x % ngroups;
+    const uint32_t b = unit / lv.H, h = unit % lv.H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long W = lv.W;
+    const long long entered_old = W ? max(0LL, (long long)n0 - W) : (long long)n0;
+    for (int r = warp; r < 32; r += 8) {
+        const long long p = 32LL * g + r;
+        float x[CPL];
+        if (p < entered_old) {
+            const float* src = lv.pend + ((long long)unit * 32 + p % 32) * D + lane * CPL;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) x[j] = src[j];
+        } else if (p < (long long)n0) {                  // leaves the ring now
+            const uint8_t* srow = lv.ring[0] + (long long)unit * lv.ring_region + (p % W) * lv.tail.stride;
+            load_row_values<CPL>(srow, lv.tail, lane, x);
+        } else {
+            const long long i = p - n0;
+            float y[CPL];
+            load_row_f32<CPL>(k + (((long long)b * C + i) * lv.H + h) * D, lane, y);
+            if (W) tail_round<CPL>(lv.tail, y, x);
+            else {
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) x[j] = y[j];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) sg[r * D + lane * CPL + j] = x[j];
+    }
+    __syncthreads();
+    const RowFmt f = lv.fmt[0];
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+        float v[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = sg[t * D + c];
+        uint32_t u[32];
+        uint16_t dh, mh = 0;
+        if (!f.asym) {
+            const int qmax = (1 << (f.bits - 1)) - 1;
+            float a = 0.f;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) a = fmaxf(a, fabsf(v[t]));
+            const float d32 = div_range(a, f.bits - 1);
+            dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
+            const float d = __half2float(__ushort_as_half(dh));
+            float t[32];
+            round_codes<32, false>(v, d, 0.f, (float)-qmax, (float)qmax, t);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = (uint32_t)(__float_as_int(t[j]) - (MAGIC_BITS - qmax - 1));
+        } else {
+            const int umax = (1 << f.bits) - 1;
+            float lo = v[0], hi = v[0];
+#pragma unroll
+            for (int t = 1; t < 32; ++t) { lo = fminf(lo, v[t]); hi = fmaxf(hi, v[t]); }
+            const float d32 = div_range(__fsub_rn(hi, lo), f.bits);
+            dh = __half_as_ushort(__float2half_rn(fminf(d32, 65504.f)));
+            mh = __half_as_ushort(__float2half_rn(fminf(fmaxf(lo, -65504.f), 65504.f)));
+            const float d = __half2float(__ushort_as_half(dh));
+            const float m = __half2float(__ushort_as_half(mh));
+            float t[32];
+            round_codes<32, true>(v, d, m, 0.f, (float)umax, t);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = (uint32_t)(__float_as_int(t[j]) - MAGIC_BITS);
+        }
+        // canonical block: d | [m] | plane0 (32 codes x w0 bits) | plane1 (32 codes x w1 bits)
+        uint16_t* blk = reinterpret_cast<uint16_t*>(lv.main[0] + (long long)unit * lv.main_region[0] +
+                                                    ((long long)g * D + c) * lv.kbb);
+        int o = 0;
+        blk[o++] = dh;
+        if (f.asym) blk[o++] = mh;
+        const int ws[2] = {f.w0, f.w1};
+        for (int pl = 0; pl < 2; ++pl) {
+            const int w = ws[pl];
+            if (w == 0) break;
+            const uint32_t mask = (1u << w) - 1;
+            const int shift = pl ? f.w0 : 0;
+            // 32 codes x w bits = 2w 16-bit words
+            for (int q = 0; q < 2 * w; ++q) {
+                uint32_t word = 0;
+                const int per = 16 / w;                  // codes per 16-bit word
+                for (int e = 0; e < per; ++e) word |= ((u[q * per + e] >> shift) & mask) << (e * w);
+                blk[o++] = (uint16_t)word;
+            }
+        }
+    }
 }
 
 // KVarN statistics: one CTA of T/2 threads per (b, h, K|V, channel group of 8);
@@ -350,11 +482,34 @@ cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, l
     const unsigned grid = (unsigned)((items + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
     const dim3 block(32 * WARPS_PER_CTA);
     const uint32_t n32 = (uint32_t)n, C32 = (uint32_t)C;
+    uint32_t done = 0;
+    if (lv.kivi) {
+        // per-channel K: quantize the groups this append completes (before the ring and the
+        // pending rows are overwritten), then the append sends the rest to the pending rows
+        const long long e0 = lv.W ? std::max(0LL, n - lv.W) : n;
+        const long long e1 = lv.W ? std::max(0LL, n + C - lv.W) : n + C;
+        const long long g0 = e0 / 32, g1 = e1 / 32;
+        done = (uint32_t)(32 * g1);
+        if (g1 > g0) {
+            const long long ng = g1 - g0;
+            const unsigned gg = (unsigned)(lv.B * lv.H * ng);
+            const size_t smem = (size_t)32 * lv.D * sizeof(float);
+            switch (lv.D / 32) {
+                case 1: kivi_group_kernel<1><<<gg, 256, smem, st>>>(lv, k, n32, C32, (uint32_t)g0, (uint32_t)ng); break;
+                case 2: kivi_group_kernel<2><<<gg, 256, smem, st>>>(lv, k, n32, C32, (uint32_t)g0, (uint32_t)ng); break;
+                case 4: kivi_group_kernel<4><<<gg, 256, smem, st>>>(lv, k, n32, C32, (uint32_t)g0, (uint32_t)ng); break;
+                case 8: kivi_group_kernel<8><<<gg, 256, smem, st>>>(lv, k, n32, C32, (uint32_t)g0, (uint32_t)ng); break;
+                default: return cudaErrorInvalidValue;
+            }
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+    }
     switch (lv.D / 32) {
-        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
-        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
-        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
-        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n32, C32); break;
+        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
+        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
+        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
+        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -40,6 +40,40 @@ struct P1Args {
     int n_idx;
 };
 
+// Per-channel K: this lane's CPL values of the K row at position pos (pos < entered, the
+// positions that have entered the K store): from the group blocks when pos's group is
+// complete, else from the pending float32 row. Dequantization as for a per-token block:
+// d * (u - 2^(X-1)) or d * u + m in float32.
+template <int CPL>
+__device__ __forceinline__ void load_kivi_k(const LayerView& lv, const uint8_t* kreg, const float* pend, long long pos,
+                                            long long entered, int lane, float (&x)[CPL]) {
+    const int D = lv.D;
+    if (pos >= entered / 32 * 32) {
+        const float* r = pend + (pos % 32) * D + lane * CPL;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) x[j] = r[j];
+        return;
+    }
+    const RowFmt f = lv.fmt[0];
+    const int t = (int)(pos % 32);
+    const int off = 1 << (f.bits - 1);
+    const int p0 = f.asym ? 4 : 2, p1 = p0 + 4 * f.w0;
+    const uint32_t m0 = (1u << f.w0) - 1, m1 = (1u << f.w1) - 1;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const uint8_t* blk = kreg + ((pos / 32) * D + lane * CPL + j) * (long long)lv.kbb;
+        const float d = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk)));
+        uint32_t u = (blk[p0 + (t * f.w0) / 8] >> ((t * f.w0) % 8)) & m0;
+        if (f.w1) u |= ((blk[p1 + (t * f.w1) / 8] >> ((t * f.w1) % 8)) & m1) << f.w0;
+        if (f.asym) {
+            const float m = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk + 2)));
+            x[j] = __fadd_rn(__fmul_rn(d, (float)u), m);
+        } else {
+            x[j] = __fmul_rn(d, (float)((int)u - off));
+        }
+    }
+}
+
 template <int CPL>
 __global__ void __launch_bounds__(32 * P1_WARPS)
 attn_pass1(P1Args a) {
@@ -112,7 +146,11 @@ attn_pass1(P1Args a) {
             if (pos > limit) continue;
         }
         float kx[CPL], vx[CPL];
-        load_row_values<CPL>(kbase + row * fk.stride, fk, lane, kx);
+        if (lv.kivi && !a.ring)
+            load_kivi_k<CPL>(lv, kbase, lv.pend + (long long)(b * H + h) * 32 * D, row,
+                             lv.W ? a.n - (a.n < lv.W ? a.n : lv.W) : a.n, lane, kx);
+        else
+            load_row_values<CPL>(kbase + row * fk.stride, fk, lane, kx);
         load_row_values<CPL>(vbase + row * fv.stride, fv, lane, vx);
         float s[MAXG];
 #pragma unroll
@@ -341,7 +379,7 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
     const long long n_ring = lv.W ? (n < lv.W ? n : (long long)lv.W) : 0;
     const long long n_main = n - n_ring;
     const int CPL = lv.D / 32;
-    const bool tcp = use_tensor_cores(lv.D);
+    const bool tcp = use_tensor_cores(lv.D) && !lv.kivi;   // per-channel K: CUDA-core path
     int launched = 0;
     // the ring pass goes first: its few short splits take their SM slots before the
     // low-bit pass fills the rest, instead of waiting for low-bit splits to retire

@@ -115,8 +115,11 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int D = 32 * NB, G = a.G, H = a.H;
-    const size_t sb = stage_bytes(a.kstride, a.vstride);
-    const size_t mb = main_bytes(a.kstride, a.vstride, D);
+    // row strides are fixed by the formats (the host passes the same values in KS,
+    // VS to size shared memory)
+    constexpr int KS = KT::stride(NB), VS = VT::stride(NB);
+    constexpr size_t sb = stage_bytes(KS, VS);
+    constexpr size_t mb = main_bytes(KS, VS, 32 * NB);
     uint8_t* stage0 = smem;
     float* pT = reinterpret_cast<float*>(smem + mb);                                   // [CWARPS][16][8]
     float4* xs = reinterpret_cast<float4*>(smem + mb + PT_BYTES);                      // [2][CWARPS][32]
@@ -181,8 +184,8 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
         const int last_rows = (int)(t1 - t0 - (long long)(n_tiles - 1) * TOK);
         if (last_rows < TOK) {
             uint8_t* st = stage0 + ((n_tiles - 1) % STAGES) * sb;
-            const int kz0 = last_rows * a.kstride, kz1 = TOK * a.kstride;
-            const int vz0 = kz1 + last_rows * a.vstride, vz1 = kz1 + TOK * a.vstride;
+            const int kz0 = last_rows * KS, kz1 = TOK * KS;
+            const int vz0 = kz1 + last_rows * VS, vz1 = kz1 + TOK * VS;
             for (int i = kz0 + threadIdx.x * 16; i < kz1; i += THREADS * 16)
                 *reinterpret_cast<uint4*>(st + i) = make_uint4(0, 0, 0, 0);
             for (int i = vz0 + threadIdx.x * 16; i < vz1; i += THREADS * 16)
@@ -238,16 +241,16 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
             if (lane == 0) {
                 gmask[s] = (uint64_t)m0 | ((uint64_t)m1 << 32);
                 const uint32_t nv = (uint32_t)(__popc(m0) + __popc(m1));
-                mbar_arrive_expect_tx(&full[s], nv * (uint32_t)(a.kstride + a.vstride));
+                mbar_arrive_expect_tx(&full[s], nv * (uint32_t)(KS + VS));
             }
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 if (v[k]) {
                     const int rr = lane + 32 * k;
-                    bulk_g2s(st + (size_t)rr * a.kstride, kreg + row[k] * a.kstride, (uint32_t)a.kstride, &full[s]);
-                    bulk_g2s(st + (size_t)TOK * a.kstride + (size_t)rr * a.vstride, vreg + row[k] * a.vstride,
-                             (uint32_t)a.vstride, &full[s]);
+                    bulk_g2s(st + (size_t)rr * KS, kreg + row[k] * KS, (uint32_t)KS, &full[s]);
+                    bulk_g2s(st + (size_t)TOK * KS + (size_t)rr * VS, vreg + row[k] * VS,
+                             (uint32_t)VS, &full[s]);
                 }
             }
             issued = it + 1;
@@ -266,11 +269,11 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                 if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) { *fault = 1; break; }
                 const long long r0 = t0 + (long long)it * TOK;
                 const int nrows = (int)min((long long)TOK, t1 - r0);
-                const uint32_t kb = (uint32_t)(nrows * a.kstride), vb = (uint32_t)(nrows * a.vstride);
+                const uint32_t kb = (uint32_t)(nrows * KS), vb = (uint32_t)(nrows * VS);
                 uint8_t* st = stage0 + s * sb;
                 mbar_arrive_expect_tx(&full[s], kb + vb);
-                bulk_g2s(st, kreg + r0 * a.kstride, kb, &full[s]);
-                bulk_g2s(st + (size_t)TOK * a.kstride, vreg + r0 * a.vstride, vb, &full[s]);
+                bulk_g2s(st, kreg + r0 * KS, kb, &full[s]);
+                bulk_g2s(st + (size_t)TOK * KS, vreg + r0 * VS, vb, &full[s]);
                 issued = it + 1;
             }
             // before the stages are reused for the final combine (or the CTA exits), every
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
             const int nrows = (int)min((long long)TOK, t1 - r0);
             if (sub0 < nrows) {                      // uniform over the pair
                 const uint8_t* kt = stage0 + s * sb;
-                const uint8_t* vt = kt + (size_t)TOK * a.kstride;
+                const uint8_t* vt = kt + (size_t)TOK * KS;
                 const uint64_t gm = gather ? gmask[s] : 0ull;
                 auto valid = [&](int rr) -> bool {
                     if (gather) return (gm >> (sub0 + rr)) & 1ull;
@@ -389,10 +392,48 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                     return true;
                 };
                 // ---------------- S^T = K Q^T over this warp's blocks
-                const uint8_t* rg = kt + (size_t)(sub0 + g) * a.kstride;
-                const uint8_t* rg8 = kt + (size_t)(sub0 + g + 8) * a.kstride;
+                const uint8_t* rg = kt + (size_t)(sub0 + g) * KS;
+                const uint8_t* rg8 = kt + (size_t)(sub0 + g + 8) * KS;
                 float sc[4] = {0.f, 0.f, 0.f, 0.f};
-                if (ok) {
+                if (ok && !KT::is_float) {
+                    // slot t of this warp's blocks of rows g and g + 8: one wide load per plane
+                    RowPieces<KF, NB, HB> kg, kg8;
+                    kg.load(rg, b0, t);
+                    kg8.load(rg8, b0, t);
+#pragma unroll
+                    for (int j = 0; j < HB; ++j) {
+                        const int bb = b0 + j;
+                        uint32_t pg[4], pg8[4];
+                        k_pairs_r<KF, NB, HB>(kg, j, pg);
+                        k_pairs_r<KF, NB, HB>(kg8, j, pg8);
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const uint32_t af[4] = {pg[2 * m], pg8[2 * m], pg[2 * m + 1], pg8[2 * m + 1]};
+#pragma unroll
+                            for (int pp = 0; pp < KP; ++pp) {
+                                const uint2 qv2 = qs[((bb * 2 + m) * KP + pp) * 32 + lane];
+                                mma_f<KF>(acc, af, qv2.x, qv2.y);
+                            }
+                        }
+                        const uint32_t dsel = (j & 1) ? 0x7632u : 0x5410u;
+                        const uint32_t dd = prmt(kg.d[j >> 1], kg8.d[j >> 1], dsel);
+                        const float2 df = __half22float2(*reinterpret_cast<const __half2*>(&dd));
+                        sc[0] = fmaf(acc[0], df.x, sc[0]);
+                        sc[1] = fmaf(acc[1], df.x, sc[1]);
+                        sc[2] = fmaf(acc[2], df.y, sc[2]);
+                        sc[3] = fmaf(acc[3], df.y, sc[3]);
+                        if constexpr (KT::asym) {
+                            const uint32_t mm = prmt(kg.m[j >> 1], kg8.m[j >> 1], dsel);
+                            const float2 mf = __half22float2(*reinterpret_cast<const __half2*>(&mm));
+                            const float2 qq = *reinterpret_cast<const float2*>(&qsum_s[bb * 8 + 2 * t]);
+                            sc[0] = fmaf(mf.x, qq.x, sc[0]);
+                            sc[1] = fmaf(mf.x, qq.y, sc[1]);
+                            sc[2] = fmaf(mf.y, qq.x, sc[2]);
+                            sc[3] = fmaf(mf.y, qq.y, sc[3]);
+                        }
+                    }
+                } else if (ok) {
 #pragma unroll
                     for (int j = 0; j < HB; ++j) {
                         const int bb = b0 + j;
@@ -492,10 +533,10 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                 pv[3] = myT[(tk2 + 1) * 8 + g];
                 __syncwarp();
                 const bool v0 = valid(tk0), v1 = valid(tk0 + 1), v2 = valid(tk2), v3 = valid(tk2 + 1);
-                const uint8_t* vr0 = vt + (size_t)(sub0 + tk0) * a.vstride;
-                const uint8_t* vr1 = vr0 + a.vstride;
-                const uint8_t* vr2 = vt + (size_t)(sub0 + tk2) * a.vstride;
-                const uint8_t* vr3 = vr2 + a.vstride;
+                const uint8_t* vr0 = vt + (size_t)(sub0 + tk0) * VS;
+                const uint8_t* vr1 = vr0 + VS;
+                const uint8_t* vr2 = vt + (size_t)(sub0 + tk2) * VS;
+                const uint8_t* vr3 = vr2 + VS;
                 // P split once per sub-tile (invalid tokens carry p = 0)
                 uint32_t bp[3][2];
                 {
@@ -506,12 +547,20 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                     for (int pp = 0; pp < 3; ++pp) { bp[pp][0] = x01[pp]; bp[pp][1] = x23[pp]; }
                 }
                 // ---------------- O^T += V^T P^T over this warp's blocks
+                // slot g >> 1 of this warp's blocks of the four rows: one wide load per plane
+                RowPieces<VF, NB, HB> vp0, vp1, vp2, vp3;
+                if constexpr (VSCALED) {
+                    vp0.load(vr0, b0, g >> 1);
+                    vp1.load(vr1, b0, g >> 1);
+                    vp2.load(vr2, b0, g >> 1);
+                    vp3.load(vr3, b0, g >> 1);
+                }
 #pragma unroll
                 for (int j = 0; j < HB; ++j) {
                     const int bb = b0 + j;
                     if constexpr (VSCALED) {
                         uint32_t ah[2][4], al[2][4];
-                        v_frags_scaled<VF>(vr0, vr1, vr2, vr3, NB, bb, g, vmul, ah, al);
+                        v_frags_scaled_r<VF, NB, HB>(vp0, vp1, vp2, vp3, j, g & 1, vmul, ah, al);
 #pragma unroll
                         for (int m = 0; m < 2; ++m) {
                             mma_f16(o[j][m], ah[m], bp[0][0], bp[0][1]);
@@ -521,14 +570,19 @@ __global__ void __launch_bounds__(THREADS, min_ctas(NB)) decode_tc(Args a) {
                         if constexpr (VT::asym) {
                             // min term of the centred codes: m + d * c (c = (2^bits - 1)/2)
                             constexpr float VC = VT::vcenter;
-                            const float m0 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr0)[bb]), VC,
-                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr0 + VT::off_m(NB))[bb]));
-                            const float m1 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr1)[bb]), VC,
-                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr1 + VT::off_m(NB))[bb]));
-                            const float m2 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr2)[bb]), VC,
-                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr2 + VT::off_m(NB))[bb]));
-                            const float m3 = fmaf(h2f_lo(reinterpret_cast<const uint16_t*>(vr3)[bb]), VC,
-                                                  h2f_lo(reinterpret_cast<const uint16_t*>(vr3 + VT::off_m(NB))[bb]));
+                            const uint32_t dsel = (j & 1) ? 0x7632u : 0x5410u;
+                            const uint32_t d01 = prmt(vp0.d[j >> 1], vp1.d[j >> 1], dsel);
+                            const uint32_t d23 = prmt(vp2.d[j >> 1], vp3.d[j >> 1], dsel);
+                            const uint32_t m01 = prmt(vp0.m[j >> 1], vp1.m[j >> 1], dsel);
+                            const uint32_t m23 = prmt(vp2.m[j >> 1], vp3.m[j >> 1], dsel);
+                            const float2 fd01 = __half22float2(*reinterpret_cast<const __half2*>(&d01));
+                            const float2 fd23 = __half22float2(*reinterpret_cast<const __half2*>(&d23));
+                            const float2 fm01 = __half22float2(*reinterpret_cast<const __half2*>(&m01));
+                            const float2 fm23 = __half22float2(*reinterpret_cast<const __half2*>(&m23));
+                            const float m0 = fmaf(fd01.x, VC, fm01.x);
+                            const float m1 = fmaf(fd01.y, VC, fm01.y);
+                            const float m2 = fmaf(fd23.x, VC, fm23.x);
+                            const float m3 = fmaf(fd23.y, VC, fm23.y);
                             float acc = pm[j];
                             if (v0) acc = fmaf(pv[0], m0, acc);
                             if (v1) acc = fmaf(pv[1], m1, acc);

@@ -17,7 +17,7 @@ struct kvq_cache {
     int kf, vf, tf, W;
     RowFmt fmt[2], tail;
     // byte offsets of the areas inside the bound buffer
-    size_t off_main[2], off_ring[2], off_scales, off_meta;
+    size_t off_main[2], off_ring[2], off_scales, off_pend, off_meta;
     size_t main_region[2], ring_region;   // bytes per (layer, b, h) region
     size_t total;
     uint8_t* buf;
@@ -56,6 +56,10 @@ LayerView layer_view(const kvq_cache* c, int layer) {
                           : nullptr;
     v.tail = c->tail;
     uint32_t* meta = reinterpret_cast<uint32_t*>(c->buf + c->off_meta);
+    v.kivi = c->L.k_per_channel;
+    v.kbb = block_bytes(c->kf);
+    v.pend = c->L.k_per_channel ? reinterpret_cast<float*>(c->buf + c->off_pend) + (size_t)layer * units * 32 * c->L.head_dim
+                                : nullptr;
     v.status = meta;
     v.stats = meta + META_HEADER_WORDS + (size_t)layer * units * 4;
     v.B = c->L.batch;
@@ -98,8 +102,10 @@ kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_f
     *out = nullptr;
     const kvq_layout& L = *layout;
     if (L.n_layers < 1 || L.batch < 1 || L.n_kv_heads < 1 || L.n_q_heads < L.n_kv_heads ||
-        L.n_q_heads % L.n_kv_heads || L.max_ctx < 1 || L.max_ctx > (1LL << 31) || L.reserved != 0)
+        L.n_q_heads % L.n_kv_heads || L.max_ctx < 1 || L.max_ctx > (1LL << 31))
         return KVQ_ERR_INVALID_ARG;
+    if (L.k_per_channel != 0 && L.k_per_channel != 1) return KVQ_ERR_INVALID_ARG;
+    if (L.k_per_channel && L.kvarn) return KVQ_ERR_INVALID_ARG;
     const int D = L.head_dim;
     if (D != 32 && D != 64 && D != 128 && D != 256) return KVQ_ERR_INVALID_ARG;
     const int G = L.n_q_heads / L.n_kv_heads;
@@ -126,6 +132,8 @@ kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_f
     size_t off = 0;
     for (int kv = 0; kv < 2; ++kv) {
         c->main_region[kv] = align_up((size_t)L.max_ctx * c->fmt[kv].stride, 256);
+        if (kv == 0 && L.k_per_channel)   // whole groups of 32 positions of D blocks
+            c->main_region[kv] = align_up((size_t)((L.max_ctx + 31) / 32) * D * block_bytes(k_fmt), 256);
         c->off_main[kv] = off;
         off += units * c->main_region[kv];
     }
@@ -136,6 +144,8 @@ kvq_status kvq_cache_create(const kvq_layout* layout, kvq_fmt k_fmt, kvq_fmt v_f
     }
     c->off_scales = off;
     if (L.kvarn) off += align_up(units * 2 * D * sizeof(float), 256);
+    c->off_pend = off;
+    if (L.k_per_channel) off += align_up(units * 32 * D * sizeof(float), 256);
     c->off_meta = off;
     off += meta_bytes(L);
     c->total = off;
@@ -271,6 +281,11 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache* c, int32_t n_query_rows, 
     const long long max_split = 2 * (per_unit < 1 ? 1 : per_unit) + 2;
     const int G = c->L.n_q_heads / c->L.n_kv_heads;
     *bytes = (size_t)units * max_split * partial_floats(G, c->L.head_dim) * sizeof(float);
+    // a prefill on the staged tensor-core path keeps its dequantized tile images here instead
+    if (!c->L.k_per_channel && prefill_staged_used(c->L.head_dim, n_query_rows, G)) {
+        const size_t img = prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx);
+        if (img > *bytes) *bytes = img;
+    }
     return KVQ_OK;
 }
 
@@ -289,7 +304,7 @@ static kvq_status attention_common(kvq_cache* c, int32_t layer, const float* q, 
     const LayerView lv = layer_view(c, layer);
     const long long n_ring = c->W ? (n < c->W ? n : c->W) : 0;
     const long long units = (long long)c->L.batch * c->L.n_kv_heads * rows;
-    const int tc_ctas = use_tensor_cores(c->L.head_dim) ? tc_ctas_per_sm(c->L.head_dim) : 0;
+    const int tc_ctas = (use_tensor_cores(c->L.head_dim) && !c->L.k_per_channel) ? tc_ctas_per_sm(c->L.head_dim) : 0;
     const SplitPlan plan = plan_splits(n - n_ring, n_ring, units, c->num_sms, tc_ctas);
     return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, rows, plan, (cudaStream_t)stream));
 }
@@ -317,7 +332,7 @@ kvq_status kvq_decode_attention_indexed(kvq_cache* c, int32_t layer, const float
     const long long list_main = (c->W == 0 || n > c->W) ? n_idx : 0;
     const long long list_ring = c->W ? n_idx : 0;
     const long long units = (long long)c->L.batch * c->L.n_kv_heads;
-    const int tc_ctas = use_tensor_cores(c->L.head_dim) ? tc_ctas_per_sm(c->L.head_dim) : 0;
+    const int tc_ctas = (use_tensor_cores(c->L.head_dim) && !c->L.k_per_channel) ? tc_ctas_per_sm(c->L.head_dim) : 0;
     const SplitPlan plan = plan_splits(list_main, list_ring, units, c->num_sms, tc_ctas);
     return cuda_status(launch_attention(lv, q, scale, out, (float*)ws, n, 1, plan, (cudaStream_t)stream, idx, n_idx));
 }
@@ -325,7 +340,7 @@ kvq_status kvq_decode_attention_indexed(kvq_cache* c, int32_t layer, const float
 kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, int32_t n_chunk, float scale,
                                  float* out, void* ws, size_t ws_bytes, void* stream) {
     if (n_chunk < 1) return KVQ_ERR_INVALID_ARG;
-    if (c && prefill_supported(c->L.head_dim)) {
+    if (c && prefill_supported(c->L.head_dim) && !c->L.k_per_channel) {
         // tensor-core path: validated like the split-K path, needs no workspace
         if (layer < 0 || layer >= c->L.n_layers || !q || !out || !ws) return KVQ_ERR_INVALID_ARG;
         if (!c->buf) return KVQ_ERR_NOT_BOUND;
@@ -337,7 +352,10 @@ kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, in
         kvq_status s = kvq_decode_workspace_bytes(c, n_chunk, &need);
         if (s != KVQ_OK) return s;
         if (ws_bytes < need) return KVQ_ERR_CAPACITY;
-        return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream));
+        const int G = c->L.n_q_heads / c->L.n_kv_heads;
+        const bool staged = prefill_staged_used(c->L.head_dim, n_chunk, G);
+        return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream,
+                                          staged ? (uint8_t*)ws : nullptr, staged ? (c->L.max_ctx + 31) / 32 : 0));
     }
     return attention_common(c, layer, q, n_chunk, scale, out, ws, ws_bytes, stream);
 }
@@ -351,6 +369,30 @@ kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32
     const RowFmt* f;
     const uint8_t* base;
     const LayerView lv = layer_view(c, layer);
+    const int D = c->L.head_dim, nb = D / 32;
+    if (kv == 0 && c->L.k_per_channel && (region == 0 || region == 2)) {
+        // per-channel K: region 0 = groups pos0.. (D canonical blocks each, stored as is),
+        // region 2 = pending slots pos0.. (float32 rows)
+        const size_t unit = (size_t)(b * c->L.n_kv_heads + h);
+        size_t per, lim;
+        const uint8_t* src;
+        if (region == 0) {
+            per = (size_t)D * block_bytes(c->kf);
+            lim = (size_t)((c->L.max_ctx + 31) / 32);
+            src = lv.main[0] + unit * c->main_region[0];
+        } else {
+            per = (size_t)D * sizeof(float);
+            lim = 32;
+            src = reinterpret_cast<const uint8_t*>(lv.pend + unit * 32 * D);
+        }
+        if ((size_t)(pos0 + count) > lim) return KVQ_ERR_INVALID_ARG;
+        if (bytes < (size_t)count * per) return KVQ_ERR_CAPACITY;
+        if (count == 0) return KVQ_OK;
+        if (cudaDeviceSynchronize() != cudaSuccess) return KVQ_ERR_CUDA;
+        if (cudaMemcpy(host_dst, src + (size_t)pos0 * per, (size_t)count * per, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        return KVQ_OK;
+    }
     if (region == 0) {
         if (pos0 + count > c->L.max_ctx) return KVQ_ERR_INVALID_ARG;
         f = &c->fmt[kv];
@@ -362,7 +404,6 @@ kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32
     } else {
         return KVQ_ERR_INVALID_ARG;
     }
-    const int D = c->L.head_dim, nb = D / 32;
     const size_t canon_row = (size_t)f->row_bytes;   // same bytes, block-major order
     if (bytes < (size_t)count * canon_row) return KVQ_ERR_CAPACITY;
     if (count == 0) return KVQ_OK;
@@ -381,8 +422,10 @@ kvq_status kvq_export_blocks(const kvq_cache* c, int32_t layer, int32_t b, int32
         for (int blk = 0; blk < nb; ++blk) {
             std::memcpy(o, row + 2 * blk, 2); o += 2;
             if (f->asym) { std::memcpy(o, row + f->off_m + 2 * blk, 2); o += 2; }
-            std::memcpy(o, row + f->off_p0 + 4 * f->w0 * blk, 4 * f->w0); o += 4 * f->w0;
-            if (f->w1) { std::memcpy(o, row + f->off_p1 + 4 * f->w1 * blk, 4 * f->w1); o += 4 * f->w1; }
+            // a block's plane bytes are its four 8-channel pieces in order
+            for (int t = 0; t < 4; ++t) { std::memcpy(o, row + f->off_p0 + piece_off(nb, blk, t, f->w0), f->w0); o += f->w0; }
+            if (f->w1)
+                for (int t = 0; t < 4; ++t) { std::memcpy(o, row + f->off_p1 + piece_off(nb, blk, t, f->w1), f->w1); o += f->w1; }
         }
     }
     return KVQ_OK;

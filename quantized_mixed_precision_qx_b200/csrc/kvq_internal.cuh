@@ -7,6 +7,7 @@
 //   K ring  [L][B][H] regions of W rows (tail format row stride)        (W > 0)
 //   V ring  [L][B][H] regions of W rows                                  (W > 0)
 //   scales  [L][B][H][2][D] float32 KVarN channel scales                 (kvarn)
+//   pending [L][B][H] 32 x D float32 rows                                 (per-channel K)
 //   meta    256-byte header (word 0: device status, bits set by a kernel whose bounded
 //           wait ran out) then stats [L][B][H][2 (K|V)][2] uint32: float bits of upper
 //           bounds of |value| over every row stored so far, [0] in the stored domain
@@ -15,10 +16,19 @@
 //           that keep 16-bit tensor-core operands inside the fp16 range.
 // A low-bit row of D channels (nb = D/32 blocks) is stored as
 //   [d: nb x fp16][m: nb x fp16, qX_1 only][plane0: D*w0/8 bytes][plane1: D*w1/8 bytes]
-// padded to 16 bytes. Each plane is the little-endian bitstream of the row's codes in
-// channel order (channel c at bits [c*w, c*w + w)), so block b of a plane is the
-// contiguous byte range [b*4w, (b+1)*4w): the canonical per-block serialisation is a
-// byte permutation of this row. A bf16 / f16 row is D x 2 bytes.
+// padded to 16 bytes. A plane holds the X-bit codes' low w0 bits (plane 0) or next w1 bits
+// (plane 1) in pieces of 8 channels: piece (b, t) = channels 32b + 8t .. 32b + 8t + 7 of
+// block b, t = 0..3, is the little-endian bitstream of those 8 codes (channel 32b + 8t + j at
+// bits [j*w, j*w + w)), w bytes long, stored at byte (t * nb + b) * w of the plane. Slot t of
+// consecutive blocks is contiguous, so a thread that handles slot t of several blocks reads
+// them with one wide load. The canonical per-block serialisation is a byte permutation of
+// this row (block b of a plane = its pieces t = 0..3 in order). A bf16 / f16 row is D x 2
+// bytes in channel order.
+// With per-channel K (token-axis blocks), the K main area of a (layer, b, h) instead holds
+// groups of 32 positions, each group D canonical blocks in channel order (block (g, c) at
+// byte (g * D + c) * block_bytes: d | [m] | plane0 | plane1, code t of the block = position
+// 32 g + t at bits [t*w, t*w + w) of each plane); positions that entered the K store but
+// whose group is not complete are float32 rows in the pending area, slot pos mod 32.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -51,6 +61,14 @@ struct RowFmt {
     int stride;    // row stride in bytes (multiple of 16)
     int row_bytes; // unpadded bytes of one row
 };
+
+// Byte offset, inside a plane of w-bit codes of a row with nb blocks, of the 8-channel
+// piece (b, t) (see the layout above).
+__host__ __device__ constexpr int piece_off(int nb, int b, int t, int w) { return (t * nb + b) * w; }
+// Bit offset, inside such a plane, of channel c's code.
+__host__ __device__ constexpr int plane_bit(int nb, int c, int w) {
+    return piece_off(nb, c >> 5, (c >> 3) & 3, w) * 8 + (c & 7) * w;
+}
 
 __host__ inline RowFmt make_rowfmt(int f, int D) {
     RowFmt r{};
@@ -91,6 +109,9 @@ struct LayerView {
     RowFmt fmt[2];         // K / V low-bit formats
     RowFmt tail;           // tail format (kind 0 = q8_0)
     uint32_t* stats;       // this layer's [B][H][2][2] value bounds (see the layout above)
+    float* pend;           // per-channel K: this layer's [B][H] pending rows (else nullptr)
+    int kivi;              // per-channel (token-axis) K blocks
+    int kbb;               // per-channel K: canonical block bytes of the K format
     uint32_t* status;      // the cache's device status word
     int B, H, D, G, W;
     int kvarn;
@@ -121,6 +142,8 @@ __host__ __device__ inline int fp16_exponent(float m, int lo, int hi) {
 // ---------------------------------------------------------------- launches
 cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
                           cudaStream_t st);
+// block bytes of a format (2 + 4X, or 4 + 4X for qX_1)
+__host__ __device__ inline int block_bytes(int f) { return (fmt_asym(f) ? 4 : 2) + 4 * fmt_bits(f); }
 cudaError_t launch_calibrate(const LayerView& lv, const float* k, const float* v, int C, int T,
                              double eps, cudaStream_t st);
 
@@ -150,8 +173,14 @@ cudaError_t launch_attention(const LayerView& lv, const float* q, float scale, f
 // Chunked prefill on tcgen05 (head_dim 128 / 256): q, out [B][C][Hq][D], n = cached
 // positions after the chunk's append.
 bool prefill_supported(int D);
+// The staged prefill (tiles dequantized once per (b, h) into a workspace image area, then
+// streamed by every M-tile CTA) runs when a head has more than one 128-row M-tile.
+bool prefill_staged_used(int D, int C, int G);
+size_t prefill_image_bytes(int B, int H, int D, long long max_ctx);
+// img: image area of prefill_image_bytes(B, H, D, img_tiles * 32) bytes, or nullptr for the
+// on-the-fly kernel
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
-                           cudaStream_t st);
+                           cudaStream_t st, uint8_t* img = nullptr, long long img_tiles = 0);
 
 // One warp waits, with the bounded wait the pipelined kernels use and a limit of limit_ns,
 // on an mbarrier that nothing ever arrives on, then records the timeout in *status.

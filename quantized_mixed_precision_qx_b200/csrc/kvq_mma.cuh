@@ -35,6 +35,12 @@ struct Fmt {
     __device__ static constexpr int off_p1(int nb) { return off_p0(nb) + 32 * nb * w0 / 8; }
     // number of B-operand parts (split of the non-code operand)
     static constexpr int parts = is_bf16 ? 3 : 2;
+    // bytes of one row of nb blocks and its 16-byte-padded stride (see kvq_internal.cuh)
+    __host__ __device__ static constexpr int row_bytes(int nb) {
+        return is_float ? 64 * nb : off_p0c(nb) + 4 * nb * (w0 + w1);
+    }
+    __host__ __device__ static constexpr int stride(int nb) { return (row_bytes(nb) + 15) & ~15; }
+    __host__ __device__ static constexpr int off_p0c(int nb) { return is_float ? 0 : 2 * nb * (asym ? 2 : 1); }
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -183,6 +189,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
         }
     }
 }
+// Non-blocking test of the phase with parity `parity` (true once it has completed).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return done != 0;
+}
 // 1-D bulk copy global -> shared (TMA engine), completion counted on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -230,17 +244,17 @@ __device__ __forceinline__ void k_pairs(const uint8_t* row, int nb, int b, int t
     constexpr int w0 = FT::w0, w1 = FT::w1;
     const uint8_t* p0 = row + FT::off_p0(nb);
     if constexpr (w0 == 4) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(p0 + 16 * b + 4 * t);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p0 + piece_off(nb, b, t, 4));
         p[0] = and_or(w, 0x000F000Fu, MAGIC);
         p[1] = and_or(w >> 4, 0x000F000Fu, MAGIC);
         p[2] = and_or(w >> 8, 0x000F000Fu, MAGIC);
         p[3] = and_or(w >> 12, 0x000F000Fu, MAGIC);
     } else if constexpr (w0 == 8) {
-        const uint2 w = *reinterpret_cast<const uint2*>(p0 + 32 * b + 8 * t);
+        const uint2 w = *reinterpret_cast<const uint2*>(p0 + piece_off(nb, b, t, 8));
 #pragma unroll
         for (int j = 0; j < 4; ++j) p[j] = and_or(prmt(w.x, w.y, (uint32_t)(j | ((4 + j) << 8))), 0x00FF00FFu, MAGIC);
     } else {  // w0 == 2
-        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p0 + 8 * b + 2 * t);
+        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p0 + piece_off(nb, b, t, 2));
         const uint32_t x = prmt(hw, 0u, 0x4140u);
         p[0] = and_or(x, 0x00030003u, MAGIC);
         p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
@@ -249,7 +263,7 @@ __device__ __forceinline__ void k_pairs(const uint8_t* row, int nb, int b, int t
     }
     if constexpr (w1 == 2) {
         const uint8_t* p1 = row + FT::off_p1(nb);
-        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p1 + 8 * b + 2 * t);
+        const uint32_t hw = *reinterpret_cast<const uint16_t*>(p1 + piece_off(nb, b, t, 2));
         const uint32_t x = prmt(hw, 0u, 0x4140u);
         constexpr uint32_t M = 0x00030003u << w0;
         p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
@@ -258,7 +272,7 @@ __device__ __forceinline__ void k_pairs(const uint8_t* row, int nb, int b, int t
         p[3] = and_or(shift<w0 - 6>(x), M, p[3]);
     } else if constexpr (w1 == 1) {
         const uint8_t* p1 = row + FT::off_p1(nb);
-        const uint32_t by = p1[4 * b + t];
+        const uint32_t by = p1[piece_off(nb, b, t, 1)];
         const uint32_t x = by | (by << 12);
         constexpr uint32_t M = 0x00010001u << w0;
         p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
@@ -320,21 +334,21 @@ __device__ __forceinline__ void v_pairs(const uint8_t* ra, const uint8_t* rb, in
     } else {
         const int o0 = FT::off_p0(nb);
         if constexpr (w0 == 4) {
-            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + 16 * b + 4 * k);
-            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + 16 * b + 4 * k);
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + piece_off(nb, b, k, 4));
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + piece_off(nb, b, k, 4));
             const uint32_t x = prmt(wa, wb, hs ? 0x7632u : 0x5410u);
             p[0] = and_or(x, 0x000F000Fu, MAGIC);
             p[1] = and_or(x >> 4, 0x000F000Fu, MAGIC);
             p[2] = and_or(x >> 8, 0x000F000Fu, MAGIC);
             p[3] = and_or(x >> 12, 0x000F000Fu, MAGIC);
         } else if constexpr (w0 == 8) {
-            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + 32 * b + 8 * k + 4 * hs);
-            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + 32 * b + 8 * k + 4 * hs);
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(ra + o0 + piece_off(nb, b, k, 8) + 4 * hs);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(rb + o0 + piece_off(nb, b, k, 8) + 4 * hs);
 #pragma unroll
             for (int i = 0; i < 4; ++i) p[i] = and_or(prmt(wa, wb, (uint32_t)(i | ((4 + i) << 8))), 0x00FF00FFu, MAGIC);
         } else {  // w0 == 2
-            const uint32_t ba = ra[o0 + 8 * b + 2 * k + hs];
-            const uint32_t bb = rb[o0 + 8 * b + 2 * k + hs];
+            const uint32_t ba = ra[o0 + piece_off(nb, b, k, 2) + hs];
+            const uint32_t bb = rb[o0 + piece_off(nb, b, k, 2) + hs];
             const uint32_t x = prmt(ba, bb, 0x5410u);
             p[0] = and_or(x, 0x00030003u, MAGIC);
             p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
@@ -343,8 +357,8 @@ __device__ __forceinline__ void v_pairs(const uint8_t* ra, const uint8_t* rb, in
         }
         if constexpr (w1 == 2) {
             const int o1 = FT::off_p1(nb);
-            const uint32_t ha = ra[o1 + 8 * b + 2 * k + hs];
-            const uint32_t hb = rb[o1 + 8 * b + 2 * k + hs];
+            const uint32_t ha = ra[o1 + piece_off(nb, b, k, 2) + hs];
+            const uint32_t hb = rb[o1 + piece_off(nb, b, k, 2) + hs];
             const uint32_t y = prmt(ha, hb, 0x5410u);
             constexpr uint32_t M = 0x00030003u << w0;
             p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
@@ -353,8 +367,8 @@ __device__ __forceinline__ void v_pairs(const uint8_t* ra, const uint8_t* rb, in
             p[3] = and_or(shift<w0 - 6>(y), M, p[3]);
         } else if constexpr (w1 == 1) {
             const int o1 = FT::off_p1(nb);
-            const uint32_t ha = ra[o1 + 4 * b + k];
-            const uint32_t hb = rb[o1 + 4 * b + k];
+            const uint32_t ha = ra[o1 + piece_off(nb, b, k, 1)];
+            const uint32_t hb = rb[o1 + piece_off(nb, b, k, 1)];
             const uint32_t y = prmt(ha, hb, 0x5410u) >> (4 * hs);
             constexpr uint32_t M = 0x00010001u << w0;
             p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
@@ -409,6 +423,208 @@ __device__ __forceinline__ void v_frags_scaled(const uint8_t* r0, const uint8_t*
     v_pairs<F>(r2, r3, nb, b, g, pb);
     const uint32_t d01 = prmt(reinterpret_cast<const uint16_t*>(r0)[b], reinterpret_cast<const uint16_t*>(r1)[b], 0x5410u);
     const uint32_t d23 = prmt(reinterpret_cast<const uint16_t*>(r2)[b], reinterpret_cast<const uint16_t*>(r3)[b], 0x5410u);
+    const __half2 vm = *reinterpret_cast<const __half2*>(&vmul);
+    const __half2 da = __hmul2_rn(*reinterpret_cast<const __half2*>(&d01), vm);
+    const __half2 db = __hmul2_rn(*reinterpret_cast<const __half2*>(&d23), vm);
+    uint32_t ha[4], la[4], hb[4], lb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 xa = *reinterpret_cast<const __half2*>(&pa[i]);
+        const __half2 xb = *reinterpret_cast<const __half2*>(&pb[i]);
+        const __half2 h1 = __hmul2_rn(xa, da);
+        const __half2 h2 = __hmul2_rn(xb, db);
+        const __half2 l1 = __hfma2(xa, da, __hneg2(h1));
+        const __half2 l2 = __hfma2(xb, db, __hneg2(h2));
+        ha[i] = *reinterpret_cast<const uint32_t*>(&h1);
+        hb[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        la[i] = *reinterpret_cast<const uint32_t*>(&l1);
+        lb[i] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        ahi[mt][0] = ha[2 * mt]; ahi[mt][1] = ha[2 * mt + 1]; ahi[mt][2] = hb[2 * mt]; ahi[mt][3] = hb[2 * mt + 1];
+        alo[mt][0] = la[2 * mt]; alo[mt][1] = la[2 * mt + 1]; alo[mt][2] = lb[2 * mt]; alo[mt][3] = lb[2 * mt + 1];
+    }
+}
+
+// ---------------------------------------------------------------- wide loads of pieces
+// BYTES bytes at p (a multiple of ALIGN, the guaranteed alignment of p) into 32-bit words
+// (BYTES < 4: the low bytes of w[0]).
+template <int BYTES, int ALIGN>
+__device__ __forceinline__ void load_bytes(const uint8_t* p, uint32_t (&w)[(BYTES + 3) / 4]) {
+    if constexpr (BYTES >= 16 && ALIGN >= 16) {
+#pragma unroll
+        for (int i = 0; i < BYTES / 16; ++i) {
+            const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else if constexpr (BYTES >= 8 && ALIGN >= 8) {
+#pragma unroll
+        for (int i = 0; i < BYTES / 8; ++i) {
+            const uint2 v = reinterpret_cast<const uint2*>(p)[i];
+            w[2 * i] = v.x; w[2 * i + 1] = v.y;
+        }
+    } else if constexpr (BYTES >= 4) {
+#pragma unroll
+        for (int i = 0; i < BYTES / 4; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+    } else if constexpr (BYTES == 2) {
+        w[0] = *reinterpret_cast<const uint16_t*>(p);
+    } else {
+        w[0] = *p;
+    }
+}
+
+// The pieces of slot t of blocks b0 .. b0 + HB - 1 of one stored row (plane 0, plane 1, the
+// block scales and, for qX_1, the mins), loaded with the widest aligned loads: slot t of
+// consecutive blocks is contiguous in each plane.
+template <int F, int NB, int HB>
+struct RowPieces {
+    using FT = Fmt<F>;
+    static constexpr int B0 = HB * FT::w0, B1 = HB * FT::w1;
+    uint32_t p0[(B0 + 3) / 4];
+    uint32_t p1[B1 > 0 ? (B1 + 3) / 4 : 1];
+    uint32_t d[(2 * HB + 3) / 4];
+    uint32_t m[FT::asym ? (2 * HB + 3) / 4 : 1];
+    // alignment of a run of `len` bytes (a power of two) at a multiple of len past offset off
+    // of a 16-byte-aligned row
+    static constexpr int run_align(int off, int len) {
+        const int a = (off % 16 == 0) ? 16 : (off % 8 == 0) ? 8 : (off % 4 == 0) ? 4 : (off % 2 == 0) ? 2 : 1;
+        const int l = len >= 16 ? 16 : len;
+        return a < l ? a : l;
+    }
+
+    // row: a 16-byte-aligned stored row; b0 = HB * (0 or 1), so each run starts at a multiple
+    // of its own length inside its plane
+    __device__ __forceinline__ void load(const uint8_t* row, int b0, int t) {
+        constexpr int o0 = FT::off_p0c(NB), o1 = o0 + 4 * NB * FT::w0;
+        load_bytes<B0, run_align(o0, B0)>(row + o0 + piece_off(NB, b0, t, FT::w0), p0);
+        if constexpr (B1 > 0) load_bytes<B1, run_align(o1, B1)>(row + o1 + piece_off(NB, b0, t, FT::w1), p1);
+        load_bytes<2 * HB, run_align(0, 2 * HB)>(row + 2 * b0, d);
+        if constexpr (FT::asym) load_bytes<2 * HB, run_align(2 * NB, 2 * HB)>(row + 2 * NB + 2 * b0, m);
+    }
+    // plane bytes of block j (0 <= j < HB) of this run
+    __device__ __forceinline__ uint32_t w0word(int j) const {   // w0 == 4: the piece's 32 bits
+        return p0[j];
+    }
+    __device__ __forceinline__ uint32_t half16(const uint32_t* w, int j) const {   // 2-byte piece j
+        return (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+    }
+    __device__ __forceinline__ uint32_t byte8(const uint32_t* w, int j) const {    // 1-byte piece j
+        return (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+    }
+    __device__ __forceinline__ uint32_t dbits(int j) const { return (d[j >> 1] >> (16 * (j & 1))) & 0xFFFFu; }
+    __device__ __forceinline__ uint32_t mbits(int j) const { return (m[j >> 1] >> (16 * (j & 1))) & 0xFFFFu; }
+};
+
+// K side: the four code pairs (n_j, n_{j+4}) of block j's piece, biased by 1024 (as k_pairs)
+template <int F, int NB, int HB>
+__device__ __forceinline__ void k_pairs_r(const RowPieces<F, NB, HB>& r, int j, uint32_t (&p)[4]) {
+    using FT = Fmt<F>;
+    constexpr int w0 = FT::w0, w1 = FT::w1;
+    if constexpr (w0 == 4) {
+        const uint32_t w = r.p0[j];
+        p[0] = and_or(w, 0x000F000Fu, MAGIC);
+        p[1] = and_or(w >> 4, 0x000F000Fu, MAGIC);
+        p[2] = and_or(w >> 8, 0x000F000Fu, MAGIC);
+        p[3] = and_or(w >> 12, 0x000F000Fu, MAGIC);
+    } else if constexpr (w0 == 8) {
+        const uint32_t wx = r.p0[2 * j], wy = r.p0[2 * j + 1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = and_or(prmt(wx, wy, (uint32_t)(i | ((4 + i) << 8))), 0x00FF00FFu, MAGIC);
+    } else {  // w0 == 2: a 2-byte piece, its bytes spread to the two halves
+        const uint32_t x = prmt(r.p0[j >> 1], 0u, (j & 1) ? 0x4342u : 0x4140u);
+        p[0] = and_or(x, 0x00030003u, MAGIC);
+        p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
+        p[2] = and_or(x >> 4, 0x00030003u, MAGIC);
+        p[3] = and_or(x >> 6, 0x00030003u, MAGIC);
+    }
+    if constexpr (w1 == 2) {
+        const uint32_t x = prmt(r.p1[j >> 1], 0u, (j & 1) ? 0x4342u : 0x4140u);
+        constexpr uint32_t M = 0x00030003u << w0;
+        p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
+        p[1] = and_or(shift<w0 - 2>(x), M, p[1]);
+        p[2] = and_or(shift<w0 - 4>(x), M, p[2]);
+        p[3] = and_or(shift<w0 - 6>(x), M, p[3]);
+    } else if constexpr (w1 == 1) {
+        const uint32_t by = (r.p1[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+        const uint32_t x = by * 4097u;                 // by | by << 12 (no carries: by < 256)
+        constexpr uint32_t M = 0x00010001u << w0;
+        p[0] = and_or(shift<w0 - 0>(x), M, p[0]);
+        p[1] = and_or(shift<w0 - 1>(x), M, p[1]);
+        p[2] = and_or(shift<w0 - 2>(x), M, p[2]);
+        p[3] = and_or(shift<w0 - 3>(x), M, p[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = debias<F>(p[i]);
+}
+
+// V side: the four channel pairs over two tokens (ra, rb) of block j, half hs of slot k's
+// piece (channels 4 hs .. 4 hs + 3 of it), biased by 1024 and debiased / centred as v_pairs
+template <int F, int NB, int HB>
+__device__ __forceinline__ void v_pairs_r(const RowPieces<F, NB, HB>& ra, const RowPieces<F, NB, HB>& rb, int j,
+                                          int hs, uint32_t (&p)[4]) {
+    using FT = Fmt<F>;
+    constexpr int w0 = FT::w0, w1 = FT::w1;
+    if constexpr (w0 == 4) {
+        const uint32_t x = prmt(ra.p0[j], rb.p0[j], hs ? 0x7632u : 0x5410u);
+        p[0] = and_or(x, 0x000F000Fu, MAGIC);
+        p[1] = and_or(x >> 4, 0x000F000Fu, MAGIC);
+        p[2] = and_or(x >> 8, 0x000F000Fu, MAGIC);
+        p[3] = and_or(x >> 12, 0x000F000Fu, MAGIC);
+    } else if constexpr (w0 == 8) {
+        const uint32_t wa = ra.p0[2 * j + hs], wb = rb.p0[2 * j + hs];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = and_or(prmt(wa, wb, (uint32_t)(i | ((4 + i) << 8))), 0x00FF00FFu, MAGIC);
+    } else {  // w0 == 2: byte hs of the 2-byte piece of each row
+        const int bsel = 2 * (j & 1) + hs;
+        const uint32_t x = prmt(ra.p0[j >> 1], rb.p0[j >> 1], (uint32_t)(bsel | ((4 + bsel) << 8)));
+        p[0] = and_or(x, 0x00030003u, MAGIC);
+        p[1] = and_or(x >> 2, 0x00030003u, MAGIC);
+        p[2] = and_or(x >> 4, 0x00030003u, MAGIC);
+        p[3] = and_or(x >> 6, 0x00030003u, MAGIC);
+    }
+    if constexpr (w1 == 2) {
+        const int bsel = 2 * (j & 1) + hs;
+        const uint32_t y = prmt(ra.p1[j >> 1], rb.p1[j >> 1], (uint32_t)(bsel | ((4 + bsel) << 8)));
+        constexpr uint32_t M = 0x00030003u << w0;
+        p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
+        p[1] = and_or(shift<w0 - 2>(y), M, p[1]);
+        p[2] = and_or(shift<w0 - 4>(y), M, p[2]);
+        p[3] = and_or(shift<w0 - 6>(y), M, p[3]);
+    } else if constexpr (w1 == 1) {
+        const int bsel = j & 3;
+        const uint32_t y = prmt(ra.p1[j >> 2], rb.p1[j >> 2], (uint32_t)(bsel | ((4 + bsel) << 8))) >> (4 * hs);
+        constexpr uint32_t M = 0x00010001u << w0;
+        p[0] = and_or(shift<w0 - 0>(y), M, p[0]);
+        p[1] = and_or(shift<w0 - 1>(y), M, p[1]);
+        p[2] = and_or(shift<w0 - 2>(y), M, p[2]);
+        p[3] = and_or(shift<w0 - 3>(y), M, p[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (FT::asym) {
+            const __half2 u2 = *reinterpret_cast<const __half2*>(&p[i]);
+            const __half2 r = __hsub2(__hsub2(u2, __float2half2_rn(1024.f)), __float2half2_rn(FT::vcenter));
+            p[i] = *reinterpret_cast<const uint32_t*>(&r);
+        } else {
+            p[i] = debias<F>(p[i]);
+        }
+    }
+}
+
+// A operand of O^T = V^T P^T for block j with the block scales (times vmul) folded in as an
+// exact fp16 hi + lo pair, from the pieces of the four rows 2t, 2t+1, 2t+8, 2t+9
+template <int F, int NB, int HB>
+__device__ __forceinline__ void v_frags_scaled_r(const RowPieces<F, NB, HB>& r0, const RowPieces<F, NB, HB>& r1,
+                                                 const RowPieces<F, NB, HB>& r2, const RowPieces<F, NB, HB>& r3,
+                                                 int j, int hs, uint32_t vmul, uint32_t (&ahi)[2][4],
+                                                 uint32_t (&alo)[2][4]) {
+    uint32_t pa[4], pb[4];
+    v_pairs_r<F, NB, HB>(r0, r1, j, hs, pa);
+    v_pairs_r<F, NB, HB>(r2, r3, j, hs, pb);
+    const uint32_t dsel = (j & 1) ? 0x7632u : 0x5410u;
+    const uint32_t d01 = prmt(r0.d[j >> 1], r1.d[j >> 1], dsel);
+    const uint32_t d23 = prmt(r2.d[j >> 1], r3.d[j >> 1], dsel);
     const __half2 vm = *reinterpret_cast<const __half2*>(&vmul);
     const __half2 da = __hmul2_rn(*reinterpret_cast<const __half2*>(&d01), vm);
     const __half2 db = __hmul2_rn(*reinterpret_cast<const __half2*>(&d23), vm);

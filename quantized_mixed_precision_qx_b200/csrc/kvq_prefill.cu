@@ -123,7 +123,8 @@ struct Raw8 {
 };
 
 // same, for a row already located (e.g. in the staging buffer) with its format
-__device__ __forceinline__ void fetch8_row(const uint8_t* row, const RowFmt f, uint32_t sel, int c0, Raw8& r) {
+__device__ __forceinline__ void fetch8_row(const uint8_t* row, const RowFmt f, uint32_t sel, int c0, int nb,
+                                           Raw8& r) {
     r.sel = sel;
     if (f.kind != 0) {
         const uint8_t* a = row + 2 * c0;                       // 16-byte aligned
@@ -136,12 +137,13 @@ __device__ __forceinline__ void fetch8_row(const uint8_t* row, const RowFmt f, u
     const uint32_t d = reinterpret_cast<const uint16_t*>(row)[blk];
     const uint32_t m = f.asym ? reinterpret_cast<const uint16_t*>(row + f.off_m)[blk] : 0u;
     r.dm = d | (m << 16);
-    const uintptr_t a0 = reinterpret_cast<uintptr_t>(row + f.off_p0 + c0 * f.w0 / 8);
+    // the 8 channels c0 .. c0 + 7 form one piece of each plane (c0 is a multiple of 8)
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(row + f.off_p0 + piece_off(nb, blk, (c0 >> 3) & 3, f.w0));
     r.w = *reinterpret_cast<const unsigned long long*>(a0 & ~(uintptr_t)7);
     r.sh0 = (uint32_t)(a0 & 7) * 8;
     r.w2 = 0;
     if (f.w1) {
-        const uintptr_t a1 = reinterpret_cast<uintptr_t>(row + f.off_p1 + c0 * f.w1 / 8);
+        const uintptr_t a1 = reinterpret_cast<uintptr_t>(row + f.off_p1 + piece_off(nb, blk, (c0 >> 3) & 3, f.w1));
         r.p1 = *reinterpret_cast<const uint16_t*>(a1 & ~(uintptr_t)1);
         r.sh1 = (uint32_t)(a1 & 1) * 8;
     } else {
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                         *reinterpret_cast<uint4*>(k_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
                     } else {
                         Raw8 rk;
-                        fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, rk);
+                        fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, NB, rk);
                         float x[8], y[8];
                         decode_raw8(kside, rk, 8 * ch, x);
 #pragma unroll
@@ -669,7 +671,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
                         uint32_t sel;
                         const uint8_t* row = srow(1, t0, tp, sel);
                         Raw8 rv;
-                        fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, rv);
+                        fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, NB, rv);
                         float x[8];
                         decode_raw8(vside, rv, 8 * cc, x);
                         const bool live = tp <= tile_limit;
@@ -815,6 +817,557 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     if (warp == 0) t5::tmem_dealloc(tmem, 512);
 }
 
+// ===========================================================================
+// Staged prefill: each K~ / V~^T tile is dequantized once per (batch, kv head) into a
+// workspace image laid out exactly as the shared-memory operand tiles, then every M-tile CTA
+// of that head streams the images with bulk copies instead of dequantizing them itself (the
+// 128-row M-tiles of one head all read the same tiles: dequantizing in each of them made the
+// prefill bound by its dequantization warps).
+//
+// Image of tile t (positions t*PN .. t*PN + PN - 1 in the transposed in-tile order
+// slot_pos, positions past the end clamped to the last cached one): K~ hi | K~ lo (each PN x D
+// fp16, 128-byte-swizzled K-major), V~^T hi | V~^T lo (each D x PN fp16, 64-byte swizzle),
+// scaled by the same powers of two 2^-ek, 2^-ev as the on-the-fly kernel.
+// ===========================================================================
+__host__ __device__ constexpr size_t tile_image_bytes(int D) { return (size_t)4 * PN * D * 2; }
+
+template <int NB>
+__global__ void __launch_bounds__(256) prefill_tiles(LayerView lv, long long n, uint8_t* img, long long img_tiles) {
+    constexpr int D = 32 * NB;
+    constexpr int CHUNKS = D / 8;
+    constexpr int KUNITS = PN * CHUNKS;
+    constexpr int VUNITS = (PN / 8) * 8 * NB;
+    constexpr int GUNITS = (PN / 8) * CHUNKS * 2;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const long long t = blockIdx.x;
+    const int t0 = (int)(t * PN);
+    const int last = (int)n - 1;
+    const SideView kside = side_view(lv, b, h, 0);
+    const SideView vside = side_view(lv, b, h, 1);
+    const int W = lv.W;
+    const int ring0 = W > 0 ? (int)n - W : (int)n;
+    const int ek = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * lv.H + h) * 2 + 0) * 2 + 1]), -120, 120);
+    const int ev = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * lv.H + h) * 2 + 1) * 2 + 1]), -120, 120);
+    const float kmul = __uint_as_float((uint32_t)(127 - ek) << 23);
+    const float vmul = __uint_as_float((uint32_t)(127 - ev) << 23);
+    uint8_t* base = img + ((long long)(b * lv.H + h) * img_tiles + t) * tile_image_bytes(D);
+    uint8_t* k_hi = base;
+    uint8_t* k_lo = base + PN * D * 2;
+    uint8_t* v_hi = base + 2 * PN * D * 2;
+    uint8_t* v_lo = base + 3 * PN * D * 2;
+    // row of position p (clamped to the last cached position): the low-bit store or the ring
+    auto grow = [&](const SideView& v, int p, uint32_t& sel) -> const uint8_t* {
+        p = min(p, last);
+        if (p < ring0) { sel = 0; return v.main + (long long)p * v.fmain.stride; }
+        sel = 1;
+        return v.ring + (long long)(p % W) * v.ftail.stride;
+    };
+    auto mode = [&](const SideView& v, int e) -> int {
+        if (e != 0) return 0;
+        const int tl = min(t0 + PN - 1, last);
+        if (tl < ring0 && !v.scales && fast_fmt(v.fmain.id)) return 1;
+        if (t0 >= ring0 && fast_fmt(v.ftail.id)) return 2;
+        return 0;
+    };
+    const int kmode = mode(kside, ek);
+    const int kfid = kmode == 1 ? kside.fmain.id : kside.ftail.id;
+    for (int u = threadIdx.x; u < KUNITS; u += blockDim.x) {
+        const int kr = u / CHUNKS, ch = u % CHUNKS;
+        uint32_t sel;
+        const uint8_t* row = grow(kside, t0 + slot_pos(kr), sel);
+        if (kmode != 0) {
+            uint32_t out[8];
+            const int cb = ch >> 2, ct = ch & 3;
+            switch (kfid) {
+                case F_Q2_0: k_chunk_fast<F_Q2_0, NB>(row, cb, ct, out); break;
+                case F_Q3_0: k_chunk_fast<F_Q3_0, NB>(row, cb, ct, out); break;
+                case F_Q4_0: k_chunk_fast<F_Q4_0, NB>(row, cb, ct, out); break;
+                case F_Q5_0: k_chunk_fast<F_Q5_0, NB>(row, cb, ct, out); break;
+                case F_Q6_0: k_chunk_fast<F_Q6_0, NB>(row, cb, ct, out); break;
+                case F_Q8_0: k_chunk_fast<F_Q8_0, NB>(row, cb, ct, out); break;
+                default: k_chunk_fast<F_F16, NB>(row, cb, ct, out); break;
+            }
+            const uint32_t off = t5::sw128_offset(kr, 8 * ch, PN);
+            *reinterpret_cast<uint4*>(k_hi + off) = make_uint4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<uint4*>(k_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
+        } else {
+            Raw8 rk;
+            fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, NB, rk);
+            float x[8], y[8];
+            decode_raw8(kside, rk, 8 * ch, x);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] *= kmul;
+            kperm8(x, y);
+            store_chunk(k_hi, k_lo, kr, 8 * ch, PN, y);
+        }
+    }
+    const int vmode = mode(vside, ev);
+    if (vmode != 0) {
+        const int vfid = vmode == 1 ? vside.fmain.id : vside.ftail.id;
+        for (int u = threadIdx.x; u < VUNITS; u += blockDim.x) {
+            const int pg = u % (PN / 8), g = (u / (PN / 8)) & 7, vb = u / (PN / 8) / 8;
+            const uint8_t* rr[8];
+            uint32_t sel;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) rr[j] = grow(vside, t0 + pg + (PN / 8) * j, sel);
+            uint32_t o[4][8];
+            switch (vfid) {
+                case F_Q2_0: v_chunk_fast<F_Q2_0, NB>(rr, vb, g, o); break;
+                case F_Q3_0: v_chunk_fast<F_Q3_0, NB>(rr, vb, g, o); break;
+                case F_Q4_0: v_chunk_fast<F_Q4_0, NB>(rr, vb, g, o); break;
+                case F_Q5_0: v_chunk_fast<F_Q5_0, NB>(rr, vb, g, o); break;
+                case F_Q6_0: v_chunk_fast<F_Q6_0, NB>(rr, vb, g, o); break;
+                case F_Q8_0: v_chunk_fast<F_Q8_0, NB>(rr, vb, g, o); break;
+                default: v_chunk_fast<F_F16, NB>(rr, vb, g, o); break;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = t5::sw64_offset(32 * vb + 4 * g + c, 8 * pg);
+                *reinterpret_cast<uint4*>(v_hi + off) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                *reinterpret_cast<uint4*>(v_lo + off) = make_uint4(o[c][4], o[c][5], o[c][6], o[c][7]);
+            }
+        }
+    } else {
+        for (int u = threadIdx.x; u < GUNITS; u += blockDim.x) {
+            const int tg = u % (PN / 8), cc = (u / (PN / 8)) % CHUNKS, e4 = u / (PN / 8) / CHUNKS;
+            float xv[8][4];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int tp = t0 + tg + (PN / 8) * j;
+                uint32_t sel;
+                const uint8_t* row = grow(vside, tp, sel);
+                Raw8 rv;
+                fetch8_row(row, sel ? vside.ftail : vside.fmain, sel, 8 * cc, NB, rv);
+                float x[8];
+                decode_raw8(vside, rv, 8 * cc, x);
+                const bool live = tp <= last;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) xv[j][e] = live ? x[4 * e4 + e] * vmul : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float y[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) y[j] = xv[j][e];
+                store_chunk64(v_hi, v_lo, 8 * cc + 4 * e4 + e, 8 * tg, y);
+            }
+        }
+    }
+}
+
+struct StagedArgs {
+    LayerView lv;
+    const float* q;
+    float* out;
+    float qscale;
+    long long n;
+    int C;
+    const uint8_t* img;           // tile images of every (b, h)
+    long long img_tiles;          // tiles per (b, h) in the image area
+};
+
+constexpr int SP_OWNERS = 4;
+constexpr int SP_THREADS = 32 * (SP_OWNERS + 1);          // 4 owner warps + the issuing warp
+
+__host__ __device__ constexpr size_t sp_smem(int D) {
+    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 2 * 2 * (size_t)PN * D * 2 /* K~ x 2 */ +
+           2 * 2 * (size_t)D * PN * 2 /* V~^T x 2 */ + 2 * (size_t)PM * PN * 2 /* P hi, lo */ + 256 /* barriers */;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
+    constexpr int D = 32 * NB;
+    constexpr uint32_t KT_BYTES = 2 * PN * D * 2, VT_BYTES = 2 * D * PN * 2;   // hi + lo
+    const LayerView& lv = a.lv;
+    extern __shared__ uint8_t raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* q_hi = sm;                              // Q hi [PM x D]; Q lo lives in TMEM
+    uint8_t* kbuf = q_hi + PM * D * 2;               // 2 x (K~ hi, K~ lo)
+    uint8_t* vbuf = kbuf + 2 * KT_BYTES;             // 2 x (V~^T hi, V~^T lo)
+    uint8_t* p_hi = vbuf + 2 * VT_BYTES;             // P [PM x PN], 64-byte swizzle
+    uint8_t* p_lo = p_hi + PM * PN * 2;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);
+    uint64_t* k_full = bars;                         // [2] K~ image landed
+    uint64_t* v_full = bars + 2;                     // [2] V~^T image landed
+    uint64_t* s_full = bars + 4;                     // [2] S of a tile in TMEM buffer t % 2
+    uint64_t* s_empty = bars + 6;                    // [2] owners have read that S buffer
+    uint64_t* k_empty = bars + 8;                    // [2] S MMAs done reading that K~ buffer
+    uint64_t* p_full = bars + 10;                    // P written
+    uint64_t* o_done = bars + 11;                    // P V~ MMAs done (V~ buffer and P free)
+    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 12);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool owner = warp < SP_OWNERS;
+    const bool issuer = warp == SP_OWNERS && lane == 0;
+    const int G = lv.G, H = lv.H;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int rows_total = a.C * G;
+    const int row0 = blockIdx.x * PM;
+    const int r = row0 + (tid & (PM - 1));
+    const bool row_ok = owner && r < rows_total;
+    const int ci = row_ok ? r / G : 0;
+    const int gi = row_ok ? r % G : 0;
+    const int n = (int)a.n;
+    const int pos0 = n - a.C;
+    const int my_limit = row_ok ? pos0 + ci : -1;
+    const int last_row = min(rows_total - 1, row0 + PM - 1);
+    const int tile_limit = pos0 + last_row / G;
+    const int first_row_limit = pos0 + row0 / G;
+    const int n_tiles = tile_limit / PN + 1;
+    const int ek = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 0) * 2 + 1]), -120, 120);
+    const int ev = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 1) * 2 + 1]), -120, 120);
+    const uint8_t* img = a.img + (long long)(b * H + h) * a.img_tiles * tile_image_bytes(D);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mma::mbar_init(&k_full[i], 1);
+            mma::mbar_init(&v_full[i], 1);
+            mma::mbar_init(&s_full[i], 1);
+            mma::mbar_init(&s_empty[i], SP_OWNERS);
+            mma::mbar_init(&k_empty[i], 1);
+        }
+        mma::mbar_init(p_full, SP_OWNERS);
+        mma::mbar_init(o_done, 1);
+        *fault_flag = 0;
+        mma::fence_mbar_init();
+    }
+    if (warp == 0) { t5::tmem_alloc(tmem_slot, 512); t5::tmem_relinquish(); }
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s = tmem;                       // S: 2 buffers x 2 channel halves x PN columns
+    const uint32_t t_qlo = tmem + 4 * PN;            // Q lo: columns [4 PN, 4 PN + D/2)
+    const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+
+    // bulk copies of a tile's K~ / V~^T images (issuing thread)
+    int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+    auto copy_k = [&](int t) {
+        uint64_t* bar = &k_full[t & 1];
+        mma::mbar_arrive_expect_tx(bar, KT_BYTES);
+        mma::bulk_g2s(kbuf + (size_t)(t & 1) * KT_BYTES, img + (size_t)t * tile_image_bytes(D), KT_BYTES, bar);
+        k_last[t & 1] = t;
+    };
+    auto copy_v = [&](int t) {
+        uint64_t* bar = &v_full[t & 1];
+        mma::mbar_arrive_expect_tx(bar, VT_BYTES);
+        mma::bulk_g2s(vbuf + (size_t)(t & 1) * VT_BYTES, img + (size_t)t * tile_image_bytes(D) + KT_BYTES, VT_BYTES, bar);
+        v_last[t & 1] = t;
+    };
+    if (issuer) {
+        copy_k(0);
+        copy_v(0);
+        if (n_tiles > 1) { copy_k(1); copy_v(1); }
+    }
+
+    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row),
+    // normalised per row by 2^-eq; scores are multiplied back by 2^(eq + ek)
+    float s_mul = 1.f;
+    if (owner) {
+        const float* qr = a.q + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        float qn = 1.f;
+        if (row_ok) {
+            float mq = 0.f;
+            for (int c = 0; c < D; c += 4) {
+                const float4 p = *reinterpret_cast<const float4*>(qr + c);
+                mq = fmaxf(mq, fmaxf(fmaxf(fabsf(p.x), fabsf(p.y)), fmaxf(fabsf(p.z), fabsf(p.w))));
+            }
+            const int eq = fp16_exponent(mq * fabsf(a.qscale), -120, 120);
+            qn = __uint_as_float((uint32_t)(127 - eq) << 23);
+            s_mul = __uint_as_float((uint32_t)(127 + eq) << 23) * __uint_as_float((uint32_t)(127 + ek) << 23);
+        }
+#pragma unroll 1
+        for (int c64 = 0; c64 < D; c64 += 64) {
+            float cols[32];
+#pragma unroll
+            for (int k0 = 0; k0 < 64; k0 += 8) {
+                float x[8], y[8];
+                if (row_ok) {
+                    const float4 p = *reinterpret_cast<const float4*>(qr + c64 + k0);
+                    const float4 v = *reinterpret_cast<const float4*>(qr + c64 + k0 + 4);
+                    x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w; x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) x[j] = (x[j] * a.qscale) * qn;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) x[j] = 0.f;
+                }
+                kperm8(x, y);
+                __align__(16) __half hh[8], ll[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) split16(y[j], hh[j], ll[j]);
+                *reinterpret_cast<uint4*>(q_hi + t5::sw128_offset(tid, c64 + k0, PM)) = *reinterpret_cast<const uint4*>(hh);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    cols[k0 / 2 + j] = __uint_as_float((uint32_t)__half_as_ushort(ll[2 * j]) |
+                                                       ((uint32_t)__half_as_ushort(ll[2 * j + 1]) << 16));
+            }
+            t5::tmem_st32(t_qlo + lane_off + c64 / 2, cols);
+        }
+        t5::fence_proxy_async();
+    }
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    auto set_fault = [&]() { *fault_flag = 1; };
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float gcorr = 1.f;
+    int s_last = -1, o_last = -1;
+
+    if (owner) {
+        // ======================= softmax: S(t) -> P(t), running max and sum of the row
+        float* const orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        for (int t = 0; t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            const int t0 = t * PN;
+            const int sb = t & 1;
+            if (!warp_wait(&s_full[sb], (t >> 1) & 1)) { set_fault(); break; }
+            t5::fence_after_sync();
+            float sv[32], sv2[32];
+            t5::tmem_ld32(t_s + 2 * PN * sb + lane_off, sv);
+            t5::tmem_ld32(t_s + 2 * PN * sb + PN + lane_off, sv2);
+            t5::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(&s_empty[sb]);
+#pragma unroll
+            for (int i = 0; i < PN; ++i) sv[i] += sv2[i];
+            if (s_mul != 1.f) {
+#pragma unroll
+                for (int i = 0; i < PN; ++i) sv[i] *= s_mul;
+            }
+            const bool full = t0 + PN - 1 <= first_row_limit;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < PN; ++i) {
+                if (!full && t0 + slot_pos(i) > my_limit) sv[i] = -INFINITY;
+                mx = fmaxf(mx, sv[i]);
+            }
+            const bool raise = mx > m_run + PF_RESCALE || (m_run == -INFINITY && mx > -INFINITY);
+            const float corr = !raise ? 1.f : ((m_run == -INFINITY) ? 0.f : mma::ex2(m_run - mx));
+            if (raise) {
+                l_run *= corr;
+                m_run = mx;
+            }
+            if (t > 0) {
+                if (!warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }
+                t5::fence_after_sync();
+            }
+            if (t > 0 && t % PF_FOLD == 0) {
+                const bool first = t == PF_FOLD;
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    float o[32];
+                    t5::tmem_ld32(t_o + lane_off + c, o);
+                    if (row_ok) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            float4 g4 = first ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                              : *reinterpret_cast<const float4*>(orow + c + i);
+                            g4.x = (g4.x * gcorr + o[i]) * corr;
+                            g4.y = (g4.y * gcorr + o[i + 1]) * corr;
+                            g4.z = (g4.z * gcorr + o[i + 2]) * corr;
+                            g4.w = (g4.w * gcorr + o[i + 3]) * corr;
+                            *reinterpret_cast<float4*>(orow + c + i) = g4;
+                        }
+                    }
+                }
+                gcorr = 1.f;
+            } else {
+                gcorr *= corr;
+                if (t > 0 && __any_sync(0xffffffffu, raise)) {
+#pragma unroll 1
+                    for (int c = 0; c < D; c += 32) {
+                        float o[32];
+                        t5::tmem_ld32(t_o + lane_off + c, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= corr;
+                        t5::tmem_st32(t_o + lane_off + c, o);
+                    }
+                }
+            }
+            float ps = 0.f;
+#pragma unroll
+            for (int i = 0; i < PN; ++i) {
+                const float p = (m_run == -INFINITY || sv[i] == -INFINITY) ? 0.f : mma::ex2(sv[i] - m_run);
+                sv[i] = p;
+                ps += p;
+            }
+#pragma unroll
+            for (int k0 = 0; k0 < PN; k0 += 8) {
+                float x8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x8[j] = sv[k0 + j];
+                store_chunk64(p_hi, p_lo, tid, k0, x8);
+            }
+            l_run += ps;
+            t5::fence_proxy_async();
+            t5::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mma::mbar_arrive(p_full);
+        }
+    } else if (issuer) {
+        // ======================= MMA issue and the image copies
+        // Order on the tensor pipe: S(t + 1) is issued before O(t), so the softmax of tile t
+        // runs while S(t + 1) executes. K~(t + 2) is fetched into S(t)'s buffer as soon as S(t)
+        // has finished (polled while waiting for P(t)); V~(t + 1) as soon as P(t) shows that
+        // P V~(t - 1) has finished.
+        const uint32_t idesc_s = t5::idesc_f16(PM, PN);
+        const uint32_t idesc_o = t5::idesc_f16(PM, D);
+        const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
+        const uint64_t dph0 = t5::desc_sw64(t5::smem_addr(p_hi)), dpl0 = t5::desc_sw64(t5::smem_addr(p_lo));
+        constexpr int KH = D / 32;                   // k-steps per channel half
+        auto issue_s = [&](int t) -> bool {
+            const int sb = t & 1;
+            bool okk = poll_wait(&k_full[sb], (t >> 1) & 1);
+            if (okk && t >= 2) okk = poll_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
+            if (!okk) return false;
+            t5::fence_after_sync();
+            const uint64_t dkh0 = t5::desc_sw128(t5::smem_addr(kbuf + (size_t)sb * KT_BYTES));
+            const uint64_t dkl0 = dkh0 + (uint64_t)((PN * D * 2) >> 4);
+            const uint32_t ts = t_s + 2 * PN * sb;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkh0 + dkk, idesc_s, (k % KH) > 0);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkl0 + dkk, idesc_s, true);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ts(ts + (k >= KH ? PN : 0), t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
+            }
+            t5::mma_commit(&s_full[sb]);
+            t5::mma_commit(&k_empty[sb]);
+            s_last = t;
+            return true;
+        };
+        bool ok = issue_s(0);
+        for (int t = 0; ok && t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            const int sb = t & 1;
+            if (t + 1 < n_tiles) {
+                ok = issue_s(t + 1);
+                if (!ok) break;
+            }
+            // wait for P(t) (bounded); fetch K~(t + 2) into buffer sb once S(t) has read it
+            bool need_k = t + 2 < n_tiles;
+            {
+                const uint64_t start = mma::global_ns();
+                for (uint32_t i = 0;; ++i) {
+                    if (need_k && mma::mbar_test(&k_empty[sb], (t >> 1) & 1)) {
+                        copy_k(t + 2);
+                        need_k = false;
+                    }
+                    if (!need_k && mma::mbar_test(p_full, t & 1)) break;
+                    if ((i & 63) == 63 && mma::global_ns() - start > 2000000000ull) { ok = false; break; }
+                }
+                if (!ok) break;
+            }
+            if (t >= 1 && t + 1 < n_tiles) copy_v(t + 1);   // P V~(t - 1) is done
+            ok = poll_wait(&v_full[sb], (t >> 1) & 1);
+            if (!ok) break;
+            t5::fence_after_sync();
+            const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(vbuf + (size_t)sb * VT_BYTES));
+            const uint64_t dvl0 = dvh0 + (uint64_t)((D * PN * 2) >> 4);
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dph0 + dk, dvh0 + dk, idesc_o, t % PF_FOLD != 0 || k > 0);
+            }
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dph0 + dk, dvl0 + dk, idesc_o, true);
+            }
+#pragma unroll
+            for (int k = 0; k < PN / 16; ++k) {
+                const uint64_t dk = (uint64_t)((k * 32) >> 4);
+                t5::mma_f16_ss(t_o, dpl0 + dk, dvh0 + dk, idesc_o, true);
+            }
+            t5::mma_commit(o_done);
+            o_last = t;
+        }
+        if (!ok) set_fault();
+    }
+
+    // ---- epilogue: O / l -> out (TMEM loads by whole owner warps; only real rows store)
+    __syncthreads();
+    if (owner && !*fault_flag) {
+        if (!warp_wait(o_done, (n_tiles - 1) & 1)) set_fault();
+        t5::fence_after_sync();
+    }
+    __syncthreads();
+    const bool any_fault = *fault_flag != 0;
+    if (owner && !any_fault) {
+        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_run : 0.f;
+        const bool folded = n_tiles > PF_FOLD;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+            float o[32];
+            t5::tmem_ld32(t_o + lane_off + c, o);
+            if (row_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 g4 = folded ? *reinterpret_cast<const float4*>(orow + c + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    g4.x = (g4.x * gcorr + o[i]) * inv;
+                    g4.y = (g4.y * gcorr + o[i + 1]) * inv;
+                    g4.z = (g4.z * gcorr + o[i + 2]) * inv;
+                    g4.w = (g4.w * gcorr + o[i + 3]) * inv;
+                    *reinterpret_cast<float4*>(orow + c + i) = g4;
+                }
+            }
+        }
+    } else if (row_ok && any_fault) {
+        if (tid == 0) atomicOr(lv.status, STATUS_WAIT_TIMEOUT);
+        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
+    }
+    if (issuer) {
+        // every copy issued must have landed, and every MMA finished, before the shared and
+        // tensor memory are released (bounded waits; immediate on the normal path)
+        for (int i = 0; i < 2; ++i) {
+            if (k_last[i] >= 0) mma::mbar_wait(&k_full[i], (k_last[i] >> 1) & 1, 50000000ull);
+            if (v_last[i] >= 0) mma::mbar_wait(&v_full[i], (v_last[i] >> 1) & 1, 50000000ull);
+        }
+        if (s_last >= 0) mma::mbar_wait(&s_full[s_last & 1], (s_last >> 1) & 1, 50000000ull);
+        if (o_last >= 0) mma::mbar_wait(o_done, o_last & 1, 50000000ull);
+    }
+    t5::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) t5::tmem_dealloc(tmem, 512);
+}
+
+template <int NB>
+cudaError_t launch_staged_nb(const StagedArgs& a, cudaStream_t st) {
+    constexpr int D = 32 * NB;
+    const LayerView& lv = a.lv;
+    // images of every tile a row of the chunk sees: positions 0 .. n - 1
+    const long long tiles = (a.n + PN - 1) / PN;
+    prefill_tiles<NB><<<dim3((unsigned)tiles, (unsigned)lv.H, (unsigned)lv.B), 256, 0, st>>>(lv, a.n, (uint8_t*)a.img,
+                                                                                             a.img_tiles);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    static bool raised = false;
+    if (!raised) {
+        e = cudaFuncSetAttribute(prefill_staged<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        raised = true;
+    }
+    const dim3 grid((unsigned)((a.C * lv.G + PM - 1) / PM), (unsigned)lv.H, (unsigned)lv.B);
+    prefill_staged<NB><<<grid, SP_THREADS, sp_smem(D), st>>>(a);
+    return cudaGetLastError();
+}
+
 template <int NB>
 cudaError_t launch_prefill_nb(PrefillArgs a, cudaStream_t st) {
     constexpr int D = 32 * NB;
@@ -842,8 +1395,28 @@ cudaError_t launch_prefill_nb(PrefillArgs a, cudaStream_t st) {
 
 bool prefill_supported(int D) { return D == 128 || D == 256; }
 
+bool prefill_staged_used(int D, int C, int G) { return prefill_supported(D) && (long long)C * G > PM; }
+
+size_t prefill_image_bytes(int B, int H, int D, long long max_ctx) {
+    return (size_t)B * H * (size_t)((max_ctx + PN - 1) / PN) * tile_image_bytes(D);
+}
+
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
-                           cudaStream_t st) {
+                           cudaStream_t st, uint8_t* img, long long img_tiles) {
+    if (img && prefill_staged_used(lv.D, C, lv.G)) {
+        StagedArgs s{};
+        s.lv = lv;
+        s.q = q;
+        s.out = out;
+        s.qscale = scale * 1.4426950408889634f;
+        s.n = n;
+        s.C = C;
+        s.img = img;
+        s.img_tiles = img_tiles;
+        if (lv.D == 256) return launch_staged_nb<8>(s, st);
+        if (lv.D == 128) return launch_staged_nb<4>(s, st);
+        return cudaErrorInvalidValue;
+    }
     PrefillArgs a{};
     a.lv = lv;
     a.q = q;

@@ -38,9 +38,12 @@ __device__ __forceinline__ void load_row_f32(const float* __restrict__ row, int 
     }
 }
 
-// Read nbits = CPL*w bits of a plane starting at bit lane*nbits.
-__device__ __forceinline__ uint64_t load_plane_bits(const uint8_t* plane, int lane, int nbits) {
-    const int bit = lane * nbits;
+// Read the CPL*w bits of a plane holding the codes of channels lane*CPL .. lane*CPL + CPL - 1
+// of a row with nb blocks (CPL <= 8: they lie inside one 8-channel piece).
+template <int CPL>
+__device__ __forceinline__ uint64_t load_plane_bits(const uint8_t* plane, int nb, int lane, int w) {
+    const int nbits = CPL * w;
+    const int bit = plane_bit(nb, lane * CPL, w);
     const uint8_t* p = plane + (bit >> 3);
     switch (nbits) {
         case 64: return *reinterpret_cast<const unsigned long long*>(p);
@@ -51,10 +54,13 @@ __device__ __forceinline__ uint64_t load_plane_bits(const uint8_t* plane, int la
     }
 }
 
-// Write nbits = CPL*w bits (value v) of a plane at bit lane*nbits. Sub-byte pieces are
-// gathered into whole bytes across lanes first (all lanes of the warp participate).
-__device__ __forceinline__ void store_plane_bits(uint8_t* plane, int lane, int nbits, uint64_t v) {
-    const int bit = lane * nbits;
+// Write the CPL*w bits (value v) of channels lane*CPL .. lane*CPL + CPL - 1 into a plane of a
+// row with nb blocks. Sub-byte pieces are gathered into whole bytes across lanes first (all
+// lanes of the warp participate; the lanes sharing a byte are consecutive).
+template <int CPL>
+__device__ __forceinline__ void store_plane_bits(uint8_t* plane, int nb, int lane, int w, uint64_t v) {
+    const int nbits = CPL * w;
+    const int bit = plane_bit(nb, lane * CPL, w);
     uint8_t* p = plane + (bit >> 3);
     if (nbits >= 8) {
         switch (nbits) {
@@ -88,8 +94,9 @@ __device__ __forceinline__ void load_row_values(const uint8_t* __restrict__ row,
     const int blk = (lane * CPL) >> 5;
     const float d = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(row)[blk]));
     const float m = f.asym ? __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(row + f.off_m)[blk])) : 0.f;
-    const uint64_t p0 = load_plane_bits(row + f.off_p0, lane, CPL * f.w0);
-    const uint64_t p1 = f.w1 ? load_plane_bits(row + f.off_p1, lane, CPL * f.w1) : 0;
+    const int nb = CPL;   // blocks per row: D / 32 = CPL
+    const uint64_t p0 = load_plane_bits<CPL>(row + f.off_p0, nb, lane, f.w0);
+    const uint64_t p1 = f.w1 ? load_plane_bits<CPL>(row + f.off_p1, nb, lane, f.w1) : 0;
     const uint32_t m0 = (1u << f.w0) - 1, m1 = (1u << f.w1) - 1;
     const int off = 1 << (f.bits - 1);
 #pragma unroll

@@ -36,7 +36,7 @@ class kvq_layout(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int32), ("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("n_q_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("kvarn", ctypes.c_int32),
                 ("max_ctx", ctypes.c_int64), ("kvarn_calib_tokens", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("kvarn_eps", ctypes.c_double)]
+                ("k_per_channel", ctypes.c_int32), ("kvarn_eps", ctypes.c_double)]
 
 
 class KVQError(RuntimeError):
@@ -197,9 +197,11 @@ class KVCache:
 
     def __init__(self, n_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, k_fmt, v_fmt,
                  tail_fmt=NONE, W=0, kvarn=0, calib=512, eps=1e-6, device="cuda", stream=None,
-                 ws_rows=1):
+                 ws_rows=1, k_per_channel=0):
         import torch
-        self.layout = kvq_layout(n_layers, batch, n_kv_heads, n_q_heads, head_dim, kvarn, max_ctx, calib, 0, eps)
+        self.layout = kvq_layout(n_layers, batch, n_kv_heads, n_q_heads, head_dim, kvarn, max_ctx, calib,
+                                 k_per_channel, eps)
+        self.k_per_channel = k_per_channel
         self.B, self.H, self.Hq, self.D, self.L = batch, n_kv_heads, n_q_heads, head_dim, n_layers
         self.k_fmt, self.v_fmt, self.tail_fmt, self.W = k_fmt, v_fmt, tail_fmt, W
         self.handle = kvq_cache_create(self.layout, k_fmt, v_fmt, tail_fmt, W)
@@ -273,7 +275,15 @@ class KVCache:
         return bb * (self.D // 32)
 
     def export(self, layer, b, h, kv, region, pos0, count):
+        """region 0: low-bit rows (per-channel K: groups of D blocks); 1: ring slots;
+        2 (per-channel K): pending slots as float32 rows."""
         import numpy as np
-        out = np.empty(count * self.row_bytes(region, kv), dtype=np.uint8)
+        if region == 2:
+            n = count * self.D * 4
+        elif region == 0 and kv == 0 and self.k_per_channel:
+            n = count * self.row_bytes(0, 0) * 32
+        else:
+            n = count * self.row_bytes(region, kv)
+        out = np.empty(n, dtype=np.uint8)
         kvq_export_blocks(self.handle, layer, b, h, kv, region, pos0, count, out)
         return out
