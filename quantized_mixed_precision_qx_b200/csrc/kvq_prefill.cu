@@ -825,9 +825,11 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
 // prefill bound by its dequantization warps).
 //
 // Image of tile t (positions t*PN .. t*PN + PN - 1 in the transposed in-tile order
-// slot_pos, positions past the end clamped to the last cached one): K~ hi | K~ lo (each PN x D
-// fp16, 128-byte-swizzled K-major), V~^T hi | V~^T lo (each D x PN fp16, 64-byte swizzle),
-// scaled by the same powers of two 2^-ek, 2^-ev as the on-the-fly kernel.
+// slot_pos, positions past the end clamped to the last cached one): K~ as one 2PN x D fp16
+// operand, 128-byte-swizzled K-major, whose rows 0 .. PN-1 are the hi parts and rows
+// PN .. 2PN-1 the lo parts of the tile's positions (so one N = 2PN MMA multiplies a Q
+// fragment by both); then V~^T hi | V~^T lo (each D x PN fp16, 64-byte swizzle); scaled by the
+// same powers of two 2^-ek, 2^-ev as the on-the-fly kernel.
 // ===========================================================================
 __host__ __device__ constexpr size_t tile_image_bytes(int D) { return (size_t)4 * PN * D * 2; }
 
@@ -851,8 +853,7 @@ __global__ void __launch_bounds__(256) prefill_tiles(LayerView lv, long long n, 
     const float kmul = __uint_as_float((uint32_t)(127 - ek) << 23);
     const float vmul = __uint_as_float((uint32_t)(127 - ev) << 23);
     uint8_t* base = img + ((long long)(b * lv.H + h) * img_tiles + t) * tile_image_bytes(D);
-    uint8_t* k_hi = base;
-    uint8_t* k_lo = base + PN * D * 2;
+    uint8_t* k_hl = base;                            // [D/64][hi rows | lo rows][128 B]
     uint8_t* v_hi = base + 2 * PN * D * 2;
     uint8_t* v_lo = base + 3 * PN * D * 2;
     // row of position p (clamped to the last cached position): the low-bit store or the ring
@@ -887,9 +888,9 @@ __global__ void __launch_bounds__(256) prefill_tiles(LayerView lv, long long n, 
                 case F_Q8_0: k_chunk_fast<F_Q8_0, NB>(row, cb, ct, out); break;
                 default: k_chunk_fast<F_F16, NB>(row, cb, ct, out); break;
             }
-            const uint32_t off = t5::sw128_offset(kr, 8 * ch, PN);
-            *reinterpret_cast<uint4*>(k_hi + off) = make_uint4(out[0], out[1], out[2], out[3]);
-            *reinterpret_cast<uint4*>(k_lo + off) = make_uint4(out[4], out[5], out[6], out[7]);
+            const uint32_t off = t5::sw128_offset(kr, 8 * ch, 2 * PN);
+            *reinterpret_cast<uint4*>(k_hl + off) = make_uint4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<uint4*>(k_hl + off + PN * 128) = make_uint4(out[4], out[5], out[6], out[7]);
         } else {
             Raw8 rk;
             fetch8_row(row, sel ? kside.ftail : kside.fmain, sel, 8 * ch, NB, rk);
@@ -898,7 +899,7 @@ __global__ void __launch_bounds__(256) prefill_tiles(LayerView lv, long long n, 
 #pragma unroll
             for (int j = 0; j < 8; ++j) x[j] *= kmul;
             kperm8(x, y);
-            store_chunk(k_hi, k_lo, kr, 8 * ch, PN, y);
+            store_chunk(k_hl, k_hl + PN * 128, kr, 8 * ch, 2 * PN, y);   // lo row PN + kr
         }
     }
     const int vmode = mode(vside, ev);
@@ -966,45 +967,70 @@ struct StagedArgs {
     long long img_tiles;          // tiles per (b, h) in the image area
 };
 
-constexpr int SP_OWNERS = 4;
-constexpr int SP_THREADS = 32 * (SP_OWNERS + 1);          // 4 owner warps + the issuing warp
-
+// Warp roles of the staged kernel: 8 softmax / epilogue warps own the 128 query rows in pairs
+// (warps w and w + 4 share TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, one row per lane: both
+// compute the row's running max from all of S, each turns its half of the tile's columns
+// into P and handles its half of the O columns), and one warp whose lane 0 issues the MMAs
+// and the bulk copies.
+constexpr int SP_OWNERS = 8;
+constexpr int SP_THREADS = 32 * (SP_OWNERS + 1);
+constexpr int SP_KBUF = 3;                                 // K~ buffers: fetched two tiles ahead
 __host__ __device__ constexpr size_t sp_smem(int D) {
-    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + 2 * 2 * (size_t)PN * D * 2 /* K~ x 2 */ +
-           2 * 2 * (size_t)D * PN * 2 /* V~^T x 2 */ + 2 * (size_t)PM * PN * 2 /* P hi, lo */ + 256 /* barriers */;
+    return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + SP_KBUF * 2 * (size_t)PN * D * 2 /* K~ */ +
+           2 * 2 * (size_t)D * PN * 2 /* V~^T x 2 */ + 256 /* barriers */ + 2 * PM * 4 /* row sums */;
+}
+
+// 3-input max (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (x0, x1) -> packed fp16 hi parts and lo parts with x = hi + lo to ~22 bits (hi: x with its
+// mantissa truncated to fp16's 11 significant bits, exact in fp16's normal range)
+__device__ __forceinline__ void split16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const float h0 = __uint_as_float(__float_as_uint(x0) & 0xFFFFE000u);
+    const float h1 = __uint_as_float(__float_as_uint(x1) & 0xFFFFE000u);
+    const __half2 hh = __floats2half2_rn(h0, h1);
+    const __half2 ll = __floats2half2_rn(x0 - h0, x1 - h1);
+    hi = *reinterpret_cast<const uint32_t*>(&hh);
+    lo = *reinterpret_cast<const uint32_t*>(&ll);
 }
 
 template <int NB>
 __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     constexpr int D = 32 * NB;
+    constexpr int DH = D / 2;                        // O columns per owner warp
     constexpr uint32_t KT_BYTES = 2 * PN * D * 2, VT_BYTES = 2 * D * PN * 2;   // hi + lo
     const LayerView& lv = a.lv;
     extern __shared__ uint8_t raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* q_hi = sm;                              // Q hi [PM x D]; Q lo lives in TMEM
-    uint8_t* kbuf = q_hi + PM * D * 2;               // 2 x (K~ hi, K~ lo)
-    uint8_t* vbuf = kbuf + 2 * KT_BYTES;             // 2 x (V~^T hi, V~^T lo)
-    uint8_t* p_hi = vbuf + 2 * VT_BYTES;             // P [PM x PN], 64-byte swizzle
-    uint8_t* p_lo = p_hi + PM * PN * 2;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(p_lo + PM * PN * 2);
-    uint64_t* k_full = bars;                         // [2] K~ image landed
-    uint64_t* v_full = bars + 2;                     // [2] V~^T image landed
-    uint64_t* s_full = bars + 4;                     // [2] S of a tile in TMEM buffer t % 2
-    uint64_t* s_empty = bars + 6;                    // [2] owners have read that S buffer
-    uint64_t* k_empty = bars + 8;                    // [2] S MMAs done reading that K~ buffer
-    uint64_t* p_full = bars + 10;                    // P written
+    uint8_t* kbuf = q_hi + PM * D * 2;               // SP_KBUF x (K~ hi, K~ lo)
+    uint8_t* vbuf = kbuf + SP_KBUF * KT_BYTES;       // 2 x (V~^T hi, V~^T lo)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(vbuf + 2 * VT_BYTES);
+    uint64_t* k_full = bars;                         // [SP_KBUF] K~ image landed
+    uint64_t* k_empty = bars + 3;                    // [SP_KBUF] S MMAs done reading that K~ buffer
+    uint64_t* v_full = bars + 6;                     // [2] V~^T image landed
+    uint64_t* s_full = bars + 8;                     // S of a tile in TMEM
+    uint64_t* s_empty = bars + 9;                    // owners have read it
+    uint64_t* p_full = bars + 10;                    // P written to TMEM
     uint64_t* o_done = bars + 11;                    // P V~ MMAs done (V~ buffer and P free)
     volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 12);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+    float* l_part = reinterpret_cast<float*>(bars + 32);   // [2][PM] row sums of the two column halves
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool owner = warp < SP_OWNERS;
     const bool issuer = warp == SP_OWNERS && lane == 0;
+    const int hf = (warp >> 2) & 1;                  // owner column half
+    const int lrow = 32 * (warp & 3) + lane;         // owner's row in the M-tile
     const int G = lv.G, H = lv.H;
     const int h = blockIdx.y, b = blockIdx.z;
     const int rows_total = a.C * G;
     const int row0 = blockIdx.x * PM;
-    const int r = row0 + (tid & (PM - 1));
+    const int r = row0 + lrow;
     const bool row_ok = owner && r < rows_total;
     const int ci = row_ok ? r / G : 0;
     const int gi = row_ok ? r % G : 0;
@@ -1020,13 +1046,13 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     const uint8_t* img = a.img + (long long)(b * H + h) * a.img_tiles * tile_image_bytes(D);
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < SP_KBUF; ++i) {
             mma::mbar_init(&k_full[i], 1);
-            mma::mbar_init(&v_full[i], 1);
-            mma::mbar_init(&s_full[i], 1);
-            mma::mbar_init(&s_empty[i], SP_OWNERS);
             mma::mbar_init(&k_empty[i], 1);
         }
+        for (int i = 0; i < 2; ++i) mma::mbar_init(&v_full[i], 1);
+        mma::mbar_init(s_full, 1);
+        mma::mbar_init(s_empty, SP_OWNERS);
         mma::mbar_init(p_full, SP_OWNERS);
         mma::mbar_init(o_done, 1);
         *fault_flag = 0;
@@ -1037,18 +1063,20 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem;                       // S: 2 buffers x 2 channel halves x PN columns
+    const uint32_t t_s = tmem;                       // S: 2 channel halves x PN columns
+    const uint32_t t_p = tmem + 2 * PN;              // P: PN/2 columns of fp16 pairs hi, then PN/2 lo
     const uint32_t t_qlo = tmem + 4 * PN;            // Q lo: columns [4 PN, 4 PN + D/2)
     const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
 
     // bulk copies of a tile's K~ / V~^T images (issuing thread)
-    int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+    int k_last[SP_KBUF] = {-1, -1, -1}, v_last[2] = {-1, -1};
     auto copy_k = [&](int t) {
-        uint64_t* bar = &k_full[t & 1];
+        const int kb = t % SP_KBUF;
+        uint64_t* bar = &k_full[kb];
         mma::mbar_arrive_expect_tx(bar, KT_BYTES);
-        mma::bulk_g2s(kbuf + (size_t)(t & 1) * KT_BYTES, img + (size_t)t * tile_image_bytes(D), KT_BYTES, bar);
-        k_last[t & 1] = t;
+        mma::bulk_g2s(kbuf + (size_t)kb * KT_BYTES, img + (size_t)t * tile_image_bytes(D), KT_BYTES, bar);
+        k_last[kb] = t;
     };
     auto copy_v = [&](int t) {
         uint64_t* bar = &v_full[t & 1];
@@ -1057,13 +1085,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         v_last[t & 1] = t;
     };
     if (issuer) {
-        copy_k(0);
+        for (int t = 0; t < SP_KBUF && t < n_tiles; ++t) copy_k(t);
         copy_v(0);
-        if (n_tiles > 1) { copy_k(1); copy_v(1); }
+        if (n_tiles > 1) copy_v(1);
     }
 
-    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (owners write their own row),
-    // normalised per row by 2^-eq; scores are multiplied back by 2^(eq + ek)
+    // ---- query rows: Q hi -> shared memory, Q lo -> TMEM (each owner warp of a pair writes
+    // its half of the channels), normalised per row by 2^-eq; scores are multiplied back by
+    // 2^(eq + ek)
     float s_mul = 1.f;
     if (owner) {
         const float* qr = a.q + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
@@ -1079,7 +1108,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             s_mul = __uint_as_float((uint32_t)(127 + eq) << 23) * __uint_as_float((uint32_t)(127 + ek) << 23);
         }
 #pragma unroll 1
-        for (int c64 = 0; c64 < D; c64 += 64) {
+        for (int c64 = hf * DH; c64 < (hf + 1) * DH; c64 += 64) {
             float cols[32];
 #pragma unroll
             for (int k0 = 0; k0 < 64; k0 += 8) {
@@ -1098,7 +1127,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
                 __align__(16) __half hh[8], ll[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) split16(y[j], hh[j], ll[j]);
-                *reinterpret_cast<uint4*>(q_hi + t5::sw128_offset(tid, c64 + k0, PM)) = *reinterpret_cast<const uint4*>(hh);
+                *reinterpret_cast<uint4*>(q_hi + t5::sw128_offset(lrow, c64 + k0, PM)) = *reinterpret_cast<const uint4*>(hh);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     cols[k0 / 2 + j] = __uint_as_float((uint32_t)__half_as_ushort(ll[2 * j]) |
@@ -1113,52 +1142,71 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     t5::fence_after_sync();
     auto set_fault = [&]() { *fault_flag = 1; };
 
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;            // l_run: this warp's column half
     float gcorr = 1.f;
     int s_last = -1, o_last = -1;
 
     if (owner) {
         // ======================= softmax: S(t) -> P(t), running max and sum of the row
         float* const orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
+        const int oc0 = hf * DH;                     // this warp's O columns [oc0, oc0 + DH)
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
             const int t0 = t * PN;
-            const int sb = t & 1;
-            if (!warp_wait(&s_full[sb], (t >> 1) & 1)) { set_fault(); break; }
+            if (!warp_wait(s_full, t & 1)) { set_fault(); break; }
             t5::fence_after_sync();
             float sv[32], sv2[32];
-            t5::tmem_ld32(t_s + 2 * PN * sb + lane_off, sv);
-            t5::tmem_ld32(t_s + 2 * PN * sb + PN + lane_off, sv2);
+            t5::tmem_ld32(t_s + lane_off, sv);
+            t5::tmem_ld32(t_s + PN + lane_off, sv2);
             t5::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mma::mbar_arrive(&s_empty[sb]);
+            if (lane == 0) mma::mbar_arrive(s_empty);
 #pragma unroll
             for (int i = 0; i < PN; ++i) sv[i] += sv2[i];
-            if (s_mul != 1.f) {
+            if (t0 + PN - 1 > first_row_limit) {     // a tile that crosses the causal edge
 #pragma unroll
-                for (int i = 0; i < PN; ++i) sv[i] *= s_mul;
+                for (int i = 0; i < PN; ++i)
+                    if (t0 + slot_pos(i) > my_limit) sv[i] = -INFINITY;
             }
-            const bool full = t0 + PN - 1 <= first_row_limit;
-            float mx = -INFINITY;
+            float m8[8];
 #pragma unroll
-            for (int i = 0; i < PN; ++i) {
-                if (!full && t0 + slot_pos(i) > my_limit) sv[i] = -INFINITY;
-                mx = fmaxf(mx, sv[i]);
-            }
+            for (int i = 0; i < 8; ++i) m8[i] = fmax3(sv[4 * i], sv[4 * i + 1], fmaxf(sv[4 * i + 2], sv[4 * i + 3]));
+            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * s_mul;
             const bool raise = mx > m_run + PF_RESCALE || (m_run == -INFINITY && mx > -INFINITY);
             const float corr = !raise ? 1.f : ((m_run == -INFINITY) ? 0.f : mma::ex2(m_run - mx));
             if (raise) {
                 l_run *= corr;
                 m_run = mx;
             }
-            if (t > 0) {
+            // this warp's half of the tile: p = 2^(s * s_mul - m) (masked entries: 2^-inf = 0)
+            float p[PN / 2];
+#pragma unroll
+            for (int j = 0; j < PN / 2; ++j) p[j] = hf ? sv[PN / 2 + j] : sv[j];
+            if (m_run == -INFINITY) {
+#pragma unroll
+                for (int j = 0; j < PN / 2; ++j) p[j] = 0.f;
+            } else {
+#pragma unroll
+                for (int j = 0; j < PN / 2; ++j) p[j] = mma::ex2(fmaf(p[j], s_mul, -m_run));
+            }
+            float ps4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ps4[i] = (p[4 * i] + p[4 * i + 1]) + (p[4 * i + 2] + p[4 * i + 3]);
+            l_run += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+            uint32_t ph[PN / 4], pl[PN / 4];
+#pragma unroll
+            for (int j = 0; j < PN / 4; ++j) split16x2(p[2 * j], p[2 * j + 1], ph[j], pl[j]);
+
+            if (t > 0) {   // P V~(t - 1) must be done before O is rescaled and P(t) written
                 if (!warp_wait(o_done, (t - 1) & 1)) { set_fault(); break; }
                 t5::fence_after_sync();
             }
             if (t > 0 && t % PF_FOLD == 0) {
+                // fold: O in TMEM holds tiles [t - PF_FOLD, t); add it to the partial in the
+                // output row, apply this tile's correction; P V~(t) then starts afresh
                 const bool first = t == PF_FOLD;
 #pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
+                for (int c = oc0; c < oc0 + DH; c += 32) {
                     float o[32];
                     t5::tmem_ld32(t_o + lane_off + c, o);
                     if (row_ok) {
@@ -1179,7 +1227,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
                 gcorr *= corr;
                 if (t > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
-                    for (int c = 0; c < D; c += 32) {
+                    for (int c = oc0; c < oc0 + DH; c += 32) {
                         float o[32];
                         t5::tmem_ld32(t_o + lane_off + c, o);
 #pragma unroll
@@ -1188,22 +1236,11 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
                     }
                 }
             }
-            float ps = 0.f;
-#pragma unroll
-            for (int i = 0; i < PN; ++i) {
-                const float p = (m_run == -INFINITY || sv[i] == -INFINITY) ? 0.f : mma::ex2(sv[i] - m_run);
-                sv[i] = p;
-                ps += p;
-            }
-#pragma unroll
-            for (int k0 = 0; k0 < PN; k0 += 8) {
-                float x8[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x8[j] = sv[k0 + j];
-                store_chunk64(p_hi, p_lo, tid, k0, x8);
-            }
-            l_run += ps;
-            t5::fence_proxy_async();
+            // P hi / lo into TMEM as the A operand of the P V~ MMAs: column j < PN/2 holds the
+            // fp16 hi parts of p[2j], p[2j + 1], column PN/2 + j their lo parts; this warp
+            // writes columns 8 hf .. 8 hf + 7 of each
+            t5::tmem_st8(t_p + lane_off + (PN / 4) * hf, ph);
+            t5::tmem_st8(t_p + lane_off + PN / 2 + (PN / 4) * hf, pl);
             t5::fence_before_sync();
             __syncwarp();
             if (lane == 0) mma::mbar_arrive(p_full);
@@ -1211,87 +1248,73 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     } else if (issuer) {
         // ======================= MMA issue and the image copies
         // Order on the tensor pipe: S(t + 1) is issued before O(t), so the softmax of tile t
-        // runs while S(t + 1) executes. K~(t + 2) is fetched into S(t)'s buffer as soon as S(t)
-        // has finished (polled while waiting for P(t)); V~(t + 1) as soon as P(t) shows that
-        // P V~(t - 1) has finished.
+        // runs while S(t + 1) executes. K~(t + 3) is fetched into S(t)'s buffer once S(t) has
+        // finished; V~(t + 1) once P(t) shows that P V~(t - 1) has finished.
         const uint32_t idesc_s = t5::idesc_f16(PM, PN);
+        const uint32_t idesc_s2 = t5::idesc_f16(PM, 2 * PN);
         const uint32_t idesc_o = t5::idesc_f16(PM, D);
         const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
-        const uint64_t dph0 = t5::desc_sw64(t5::smem_addr(p_hi)), dpl0 = t5::desc_sw64(t5::smem_addr(p_lo));
-        constexpr int KH = D / 32;                   // k-steps per channel half
+        // S' = [Q hi K~hi | Q hi K~lo + Q lo K~hi] in TMEM columns [0, PN) | [PN, 2 PN): the large
+        // products accumulate alone, the two small ones in their own columns; the owners add
+        // the halves
         auto issue_s = [&](int t) -> bool {
-            const int sb = t & 1;
-            bool okk = poll_wait(&k_full[sb], (t >> 1) & 1);
-            if (okk && t >= 2) okk = poll_wait(&s_empty[sb], ((t >> 1) - 1) & 1);
+            const int kb = t % SP_KBUF;
+            bool okk = poll_wait(&k_full[kb], (t / SP_KBUF) & 1);
+            if (okk && t >= 1) okk = poll_wait(s_empty, (t - 1) & 1);   // the owners have read S(t - 1)
             if (!okk) return false;
             t5::fence_after_sync();
-            const uint64_t dkh0 = t5::desc_sw128(t5::smem_addr(kbuf + (size_t)sb * KT_BYTES));
-            const uint64_t dkl0 = dkh0 + (uint64_t)((PN * D * 2) >> 4);
-            const uint32_t ts = t_s + 2 * PN * sb;
+            const uint64_t dk0 = t5::desc_sw128(t5::smem_addr(kbuf + (size_t)kb * KT_BYTES));
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
-                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkh0 + dkk, idesc_s, (k % KH) > 0);
+                const uint64_t dq = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ss(t_s, dq0 + dq, dk0 + dkk, idesc_s2, k > 0);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                const uint64_t dk = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
-                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ss(ts + (k >= KH ? PN : 0), dq0 + dk, dkl0 + dkk, idesc_s, true);
+                const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ts(t_s + PN, t_qlo + 8 * k, dk0 + dkk, idesc_s, true);
             }
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint64_t dkk = (uint64_t)(((k >> 2) * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ts(ts + (k >= KH ? PN : 0), t_qlo + 8 * k, dkh0 + dkk, idesc_s, true);
-            }
-            t5::mma_commit(&s_full[sb]);
-            t5::mma_commit(&k_empty[sb]);
+            t5::mma_commit(s_full);
+            t5::mma_commit(&k_empty[kb]);
             s_last = t;
             return true;
         };
         bool ok = issue_s(0);
         for (int t = 0; ok && t < n_tiles; ++t) {
             if (*fault_flag) break;
-            const int sb = t & 1;
             if (t + 1 < n_tiles) {
                 ok = issue_s(t + 1);
                 if (!ok) break;
             }
-            // wait for P(t) (bounded); fetch K~(t + 2) into buffer sb once S(t) has read it
-            bool need_k = t + 2 < n_tiles;
-            {
-                const uint64_t start = mma::global_ns();
-                for (uint32_t i = 0;; ++i) {
-                    if (need_k && mma::mbar_test(&k_empty[sb], (t >> 1) & 1)) {
-                        copy_k(t + 2);
-                        need_k = false;
-                    }
-                    if (!need_k && mma::mbar_test(p_full, t & 1)) break;
-                    if ((i & 63) == 63 && mma::global_ns() - start > 2000000000ull) { ok = false; break; }
-                }
+            if (t + SP_KBUF < n_tiles) {             // S(t) has read its K~ buffer: fetch tile t + 3
+                ok = poll_wait(&k_empty[t % SP_KBUF], (t / SP_KBUF) & 1);
                 if (!ok) break;
+                copy_k(t + SP_KBUF);
             }
+            ok = poll_wait(p_full, t & 1);
+            if (!ok) break;
             if (t >= 1 && t + 1 < n_tiles) copy_v(t + 1);   // P V~(t - 1) is done
-            ok = poll_wait(&v_full[sb], (t >> 1) & 1);
+            ok = poll_wait(&v_full[t & 1], (t >> 1) & 1);
             if (!ok) break;
             t5::fence_after_sync();
-            const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(vbuf + (size_t)sb * VT_BYTES));
+            const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(vbuf + (size_t)(t & 1) * VT_BYTES));
             const uint64_t dvl0 = dvh0 + (uint64_t)((D * PN * 2) >> 4);
+            // A operand (P hi / lo) from TMEM: 8 columns per 16-position k-step
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
                 const uint64_t dk = (uint64_t)((k * 32) >> 4);
-                t5::mma_f16_ss(t_o, dph0 + dk, dvh0 + dk, idesc_o, t % PF_FOLD != 0 || k > 0);
+                t5::mma_f16_ts(t_o, t_p + 8 * k, dvh0 + dk, idesc_o, t % PF_FOLD != 0 || k > 0);
             }
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
                 const uint64_t dk = (uint64_t)((k * 32) >> 4);
-                t5::mma_f16_ss(t_o, dph0 + dk, dvl0 + dk, idesc_o, true);
+                t5::mma_f16_ts(t_o, t_p + 8 * k, dvl0 + dk, idesc_o, true);
             }
 #pragma unroll
             for (int k = 0; k < PN / 16; ++k) {
                 const uint64_t dk = (uint64_t)((k * 32) >> 4);
-                t5::mma_f16_ss(t_o, dpl0 + dk, dvh0 + dk, idesc_o, true);
+                t5::mma_f16_ts(t_o, t_p + PN / 2 + 8 * k, dvh0 + dk, idesc_o, true);
             }
             t5::mma_commit(o_done);
             o_last = t;
@@ -1300,6 +1323,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     }
 
     // ---- epilogue: O / l -> out (TMEM loads by whole owner warps; only real rows store)
+    if (owner) l_part[hf * PM + lrow] = l_run;
     __syncthreads();
     if (owner && !*fault_flag) {
         if (!warp_wait(o_done, (n_tiles - 1) & 1)) set_fault();
@@ -1309,10 +1333,11 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     const bool any_fault = *fault_flag != 0;
     if (owner && !any_fault) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
-        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_run : 0.f;
+        const float l_row = l_part[lrow] + l_part[PM + lrow];   // both column halves
+        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_row : 0.f;
         const bool folded = n_tiles > PF_FOLD;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = hf * DH; c < (hf + 1) * DH; c += 32) {
             float o[32];
             t5::tmem_ld32(t_o + lane_off + c, o);
             if (row_ok) {
@@ -1330,16 +1355,16 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     } else if (row_ok && any_fault) {
         if (tid == 0) atomicOr(lv.status, STATUS_WAIT_TIMEOUT);
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
-        for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
+        for (int c = hf * DH; c < (hf + 1) * DH; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
     if (issuer) {
         // every copy issued must have landed, and every MMA finished, before the shared and
         // tensor memory are released (bounded waits; immediate on the normal path)
-        for (int i = 0; i < 2; ++i) {
-            if (k_last[i] >= 0) mma::mbar_wait(&k_full[i], (k_last[i] >> 1) & 1, 50000000ull);
+        for (int i = 0; i < SP_KBUF; ++i)
+            if (k_last[i] >= 0) mma::mbar_wait(&k_full[i], (k_last[i] / SP_KBUF) & 1, 50000000ull);
+        for (int i = 0; i < 2; ++i)
             if (v_last[i] >= 0) mma::mbar_wait(&v_full[i], (v_last[i] >> 1) & 1, 50000000ull);
-        }
-        if (s_last >= 0) mma::mbar_wait(&s_full[s_last & 1], (s_last >> 1) & 1, 50000000ull);
+        if (s_last >= 0) mma::mbar_wait(s_full, s_last & 1, 50000000ull);
         if (o_last >= 0) mma::mbar_wait(o_done, o_last & 1, 50000000ull);
     }
     t5::fence_before_sync();
