@@ -970,10 +970,11 @@ struct StagedArgs {
 // Warp roles of the staged kernel: 8 softmax / epilogue warps own the 128 query rows in pairs
 // (warps w and w + 4 share TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, one row per lane: both
 // compute the row's running max from all of S, each turns its half of the tile's columns
-// into P and handles its half of the O columns), and one warp whose lane 0 issues the MMAs
-// and the bulk copies.
+// into P and handles its half of the O columns), one warp whose lane 0 issues the MMAs and
+// one whose lane 0 issues the bulk copies. MMA issue stalls while the tensor pipe's short
+// queue is full, so the issuing thread does nothing else that could let the queue run dry.
 constexpr int SP_OWNERS = 8;
-constexpr int SP_THREADS = 32 * (SP_OWNERS + 1);
+constexpr int SP_THREADS = 32 * (SP_OWNERS + 2);
 constexpr int SP_KBUF = 3;                                 // K~ buffers: fetched two tiles ahead
 __host__ __device__ constexpr size_t sp_smem(int D) {
     return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + SP_KBUF * 2 * (size_t)PN * D * 2 /* K~ */ +
@@ -1016,14 +1017,16 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     uint64_t* s_full = bars + 8;                     // S of a tile in TMEM
     uint64_t* s_empty = bars + 9;                    // owners have read it
     uint64_t* p_full = bars + 10;                    // P written to TMEM
-    uint64_t* o_done = bars + 11;                    // P V~ MMAs done (V~ buffer and P free)
-    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 12);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+    uint64_t* o_done = bars + 11;                    // P V~ MMAs done (P free, O readable)
+    uint64_t* v_empty = bars + 12;                   // [2] P V~ MMAs done reading that V~ buffer
+    volatile int* fault_flag = reinterpret_cast<volatile int*>(bars + 14);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
     float* l_part = reinterpret_cast<float*>(bars + 32);   // [2][PM] row sums of the two column halves
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool owner = warp < SP_OWNERS;
     const bool issuer = warp == SP_OWNERS && lane == 0;
+    const bool copier = warp == SP_OWNERS + 1 && lane == 0;
     const int hf = (warp >> 2) & 1;                  // owner column half
     const int lrow = 32 * (warp & 3) + lane;         // owner's row in the M-tile
     const int G = lv.G, H = lv.H;
@@ -1050,7 +1053,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             mma::mbar_init(&k_full[i], 1);
             mma::mbar_init(&k_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) mma::mbar_init(&v_full[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mma::mbar_init(&v_full[i], 1);
+            mma::mbar_init(&v_empty[i], 1);
+        }
         mma::mbar_init(s_full, 1);
         mma::mbar_init(s_empty, SP_OWNERS);
         mma::mbar_init(p_full, SP_OWNERS);
@@ -1063,13 +1069,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem;                       // S: 2 channel halves x PN columns
+    const uint32_t t_s = tmem;                       // S': Q hi K~hi | Q hi K~lo, PN columns each
     const uint32_t t_p = tmem + 2 * PN;              // P: PN/2 columns of fp16 pairs hi, then PN/2 lo
+    const uint32_t t_s3 = tmem + 3 * PN;             // S'': Q lo K~hi
     const uint32_t t_qlo = tmem + 4 * PN;            // Q lo: columns [4 PN, 4 PN + D/2)
     const uint32_t t_o = tmem + 256;                 // O: columns [256, 256 + D)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
 
-    // bulk copies of a tile's K~ / V~^T images (issuing thread)
+    // bulk copies of a tile's K~ / V~^T images (copying thread)
     int k_last[SP_KBUF] = {-1, -1, -1}, v_last[2] = {-1, -1};
     auto copy_k = [&](int t) {
         const int kb = t % SP_KBUF;
@@ -1084,7 +1091,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         mma::bulk_g2s(vbuf + (size_t)(t & 1) * VT_BYTES, img + (size_t)t * tile_image_bytes(D) + KT_BYTES, VT_BYTES, bar);
         v_last[t & 1] = t;
     };
-    if (issuer) {
+    if (copier) {
         for (int t = 0; t < SP_KBUF && t < n_tiles; ++t) copy_k(t);
         copy_v(0);
         if (n_tiles > 1) copy_v(1);
@@ -1155,14 +1162,15 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             const int t0 = t * PN;
             if (!warp_wait(s_full, t & 1)) { set_fault(); break; }
             t5::fence_after_sync();
-            float sv[32], sv2[32];
+            float sv[32], sv2[32], sv3[32];
             t5::tmem_ld32(t_s + lane_off, sv);
             t5::tmem_ld32(t_s + PN + lane_off, sv2);
+            t5::tmem_ld32(t_s3 + lane_off, sv3);
             t5::fence_before_sync();
             __syncwarp();
             if (lane == 0) mma::mbar_arrive(s_empty);
 #pragma unroll
-            for (int i = 0; i < PN; ++i) sv[i] += sv2[i];
+            for (int i = 0; i < PN; ++i) sv[i] += sv2[i] + sv3[i];
             if (t0 + PN - 1 > first_row_limit) {     // a tile that crosses the causal edge
 #pragma unroll
                 for (int i = 0; i < PN; ++i)
@@ -1246,17 +1254,16 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             if (lane == 0) mma::mbar_arrive(p_full);
         }
     } else if (issuer) {
-        // ======================= MMA issue and the image copies
-        // Order on the tensor pipe: S(t + 1) is issued before O(t), so the softmax of tile t
-        // runs while S(t + 1) executes. K~(t + 3) is fetched into S(t)'s buffer once S(t) has
-        // finished; V~(t + 1) once P(t) shows that P V~(t - 1) has finished.
+        // ======================= MMA issue
+        // Pipe order: S(t + 1), then O(t) once P(t) is written; the softmax of tile t runs
+        // while S(t + 1) executes.
         const uint32_t idesc_s = t5::idesc_f16(PM, PN);
         const uint32_t idesc_s2 = t5::idesc_f16(PM, 2 * PN);
         const uint32_t idesc_o = t5::idesc_f16(PM, D);
         const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
-        // S' = [Q hi K~hi | Q hi K~lo + Q lo K~hi] in TMEM columns [0, PN) | [PN, 2 PN): the large
-        // products accumulate alone, the two small ones in their own columns; the owners add
-        // the halves
+        // S' = [Q hi K~hi | Q hi K~lo] in TMEM columns [0, 2 PN), S'' = Q lo K~hi in
+        // [3 PN, 4 PN): the large products accumulate alone; the owners add the three. The short
+        // S'' MMAs go first, so the queue holds the long ones when the issue returns.
         auto issue_s = [&](int t) -> bool {
             const int kb = t % SP_KBUF;
             bool okk = poll_wait(&k_full[kb], (t / SP_KBUF) & 1);
@@ -1266,14 +1273,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             const uint64_t dk0 = t5::desc_sw128(t5::smem_addr(kbuf + (size_t)kb * KT_BYTES));
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                const uint64_t dq = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
                 const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ss(t_s, dq0 + dq, dk0 + dkk, idesc_s2, k > 0);
+                t5::mma_f16_ts(t_s3, t_qlo + 8 * k, dk0 + dkk, idesc_s, k > 0);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dq = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
                 const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ts(t_s + PN, t_qlo + 8 * k, dk0 + dkk, idesc_s, true);
+                t5::mma_f16_ss(t_s, dq0 + dq, dk0 + dkk, idesc_s2, k > 0);
             }
             t5::mma_commit(s_full);
             t5::mma_commit(&k_empty[kb]);
@@ -1287,15 +1294,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
                 ok = issue_s(t + 1);
                 if (!ok) break;
             }
-            if (t + SP_KBUF < n_tiles) {             // S(t) has read its K~ buffer: fetch tile t + 3
-                ok = poll_wait(&k_empty[t % SP_KBUF], (t / SP_KBUF) & 1);
-                if (!ok) break;
-                copy_k(t + SP_KBUF);
-            }
             ok = poll_wait(p_full, t & 1);
-            if (!ok) break;
-            if (t >= 1 && t + 1 < n_tiles) copy_v(t + 1);   // P V~(t - 1) is done
-            ok = poll_wait(&v_full[t & 1], (t >> 1) & 1);
+            if (ok) ok = poll_wait(&v_full[t & 1], (t >> 1) & 1);
             if (!ok) break;
             t5::fence_after_sync();
             const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(vbuf + (size_t)(t & 1) * VT_BYTES));
@@ -1317,7 +1317,26 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
                 t5::mma_f16_ts(t_o, t_p + PN / 2 + 8 * k, dvh0 + dk, idesc_o, true);
             }
             t5::mma_commit(o_done);
+            t5::mma_commit(&v_empty[t & 1]);
             o_last = t;
+        }
+        if (!ok) set_fault();
+    } else if (copier) {
+        // ======================= image copies: K~(t + 3) into S(t)'s buffer once S(t) has
+        // finished, V~(t + 1) into O(t - 1)'s buffer once O(t - 1) has finished
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            if (*fault_flag) break;
+            if (t + SP_KBUF < n_tiles) {
+                ok = poll_wait(&k_empty[t % SP_KBUF], (t / SP_KBUF) & 1);
+                if (!ok) break;
+                copy_k(t + SP_KBUF);
+            }
+            if (t >= 1 && t + 1 < n_tiles) {
+                ok = poll_wait(&v_empty[(t - 1) & 1], ((t - 1) >> 1) & 1);
+                if (!ok) break;
+                copy_v(t + 1);
+            }
         }
         if (!ok) set_fault();
     }
@@ -1357,15 +1376,23 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = hf * DH; c < (hf + 1) * DH; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
-    if (issuer) {
-        // every copy issued must have landed, and every MMA finished, before the shared and
-        // tensor memory are released (bounded waits; immediate on the normal path)
+    // every copy issued must have landed, and every MMA finished, before the shared and
+    // tensor memory are released (bounded waits; immediate on the normal path)
+    if (copier) {
         for (int i = 0; i < SP_KBUF; ++i)
             if (k_last[i] >= 0) mma::mbar_wait(&k_full[i], (k_last[i] / SP_KBUF) & 1, 50000000ull);
         for (int i = 0; i < 2; ++i)
             if (v_last[i] >= 0) mma::mbar_wait(&v_full[i], (v_last[i] >> 1) & 1, 50000000ull);
-        if (s_last >= 0) mma::mbar_wait(s_full, s_last & 1, 50000000ull);
-        if (o_last >= 0) mma::mbar_wait(o_done, o_last & 1, 50000000ull);
+    }
+    if (issuer) {   // the later commits of each group too (their arrivals must land first)
+        if (s_last >= 0) {
+            mma::mbar_wait(s_full, s_last & 1, 50000000ull);
+            mma::mbar_wait(&k_empty[s_last % SP_KBUF], (s_last / SP_KBUF) & 1, 50000000ull);
+        }
+        if (o_last >= 0) {
+            mma::mbar_wait(o_done, o_last & 1, 50000000ull);
+            mma::mbar_wait(&v_empty[o_last & 1], (o_last >> 1) & 1, 50000000ull);
+        }
     }
     t5::fence_before_sync();
     __syncthreads();
