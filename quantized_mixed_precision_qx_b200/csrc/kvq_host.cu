@@ -284,7 +284,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache* c, int32_t n_query_rows, 
     // a prefill on the staged tensor-core path keeps its dequantized tile images here instead
     if (!c->L.k_per_channel && prefill_staged_used(c->L.head_dim, n_query_rows, G)) {
         const size_t img = prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx);
-        if (img > *bytes) *bytes = img;
+        const size_t all = align_up(img, 256) + prefill_partial_bytes(c->L.batch, c->L.n_q_heads, c->L.head_dim,
+                                                                 n_query_rows);
+        if (all > *bytes) *bytes = all;
     }
     return KVQ_OK;
 }
@@ -354,8 +356,12 @@ kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, in
         if (ws_bytes < need) return KVQ_ERR_CAPACITY;
         const int G = c->L.n_q_heads / c->L.n_kv_heads;
         const bool staged = prefill_staged_used(c->L.head_dim, n_chunk, G);
+        if (!staged)
+            return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream));
+        const size_t img = prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx);
         return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream,
-                                          staged ? (uint8_t*)ws : nullptr, staged ? (c->L.max_ctx + 31) / 32 : 0));
+                                          (uint8_t*)ws, (c->L.max_ctx + 31) / 32,
+                                          (float*)((uint8_t*)ws + align_up(img, 256)), c->num_sms));
     }
     return attention_common(c, layer, q, n_chunk, scale, out, ws, ws_bytes, stream);
 }

@@ -24,6 +24,8 @@
 // 2 x 32 x D x 2 B per K~ tile (K-major, 128-byte swizzle), V~^T hi/lo 2 x D x 32 x 2 B and
 // P hi/lo 2 x 128 x 32 x 2 B (K-major, 64-byte swizzle), 2 staging buffers of 2 x 32 raw rows
 // (sized by the widest row format).
+#include <algorithm>
+
 #include "kvq_internal.cuh"
 #include "kvq_mma.cuh"
 #include "kvq_tc5.cuh"
@@ -39,6 +41,7 @@ constexpr float PF_RESCALE = 8.0f;
 // with IEEE fp32 adds and the next P V~ starts a fresh accumulation: long accumulation runs
 // in tensor memory lose precision (over 100k positions the error grows past 1e-4).
 constexpr int PF_FOLD = 128;
+constexpr int PF_MAX_SPLITS = 4;   // key-range splits of a staged prefill M-tile
 
 struct PrefillArgs {
     LayerView lv;
@@ -965,6 +968,9 @@ struct StagedArgs {
     int C;
     const uint8_t* img;           // tile images of every (b, h)
     long long img_tiles;          // tiles per (b, h) in the image area
+    int splits;                   // key-range splits per M-tile (1: rows finished in place)
+    float* part;                  // splits > 1: [splits][B * C * Hq][D] unnormalised O, then
+                                  // [splits][B * C * Hq][2] (running max, row sum)
 };
 
 // Warp roles of the staged kernel: 8 softmax / epilogue warps own the 128 query rows in pairs
@@ -1030,7 +1036,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     const int hf = (warp >> 2) & 1;                  // owner column half
     const int lrow = 32 * (warp & 3) + lane;         // owner's row in the M-tile
     const int G = lv.G, H = lv.H;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = blockIdx.z / a.splits, sp = blockIdx.z % a.splits;
     const int rows_total = a.C * G;
     const int row0 = blockIdx.x * PM;
     const int r = row0 + lrow;
@@ -1043,10 +1049,19 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     const int last_row = min(rows_total - 1, row0 + PM - 1);
     const int tile_limit = pos0 + last_row / G;
     const int first_row_limit = pos0 + row0 / G;
-    const int n_tiles = tile_limit / PN + 1;
+    // this CTA's key tiles: [t_lo, t_lo + n_tiles) of the M-tile's tiles_all (every split has
+    // at least one: the host splits only when the first M-tile sees splits x 32 tiles or more);
+    // the loops below count tiles from t_lo
+    const int tiles_all = tile_limit / PN + 1;
+    const int t_lo = (int)((long long)tiles_all * sp / a.splits);
+    const int n_tiles = (int)((long long)tiles_all * (sp + 1) / a.splits) - t_lo;
     const int ek = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 0) * 2 + 1]), -120, 120);
     const int ev = fp16_exponent(__uint_as_float(lv.stats[((long long)(b * H + h) * 2 + 1) * 2 + 1]), -120, 120);
-    const uint8_t* img = a.img + (long long)(b * H + h) * a.img_tiles * tile_image_bytes(D);
+    const uint8_t* img = a.img + ((long long)(b * H + h) * a.img_tiles + t_lo) * tile_image_bytes(D);
+    const long long rows_all = (long long)lv.B * a.C * G * H;
+    const long long orow_idx = ((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi;
+    // where the row's O goes: the output row, or this split's partial
+    float* const orow = a.splits > 1 ? a.part + ((long long)sp * rows_all + orow_idx) * D : a.out + orow_idx * D;
 
     if (tid == 0) {
         for (int i = 0; i < SP_KBUF; ++i) {
@@ -1155,11 +1170,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
 
     if (owner) {
         // ======================= softmax: S(t) -> P(t), running max and sum of the row
-        float* const orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         const int oc0 = hf * DH;                     // this warp's O columns [oc0, oc0 + DH)
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
-            const int t0 = t * PN;
+            const int t0 = (t_lo + t) * PN;
             if (!warp_wait(s_full, t & 1)) { set_fault(); break; }
             t5::fence_after_sync();
             float sv[32], sv2[32], sv3[32];
@@ -1351,9 +1365,15 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     __syncthreads();
     const bool any_fault = *fault_flag != 0;
     if (owner && !any_fault) {
-        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         const float l_row = l_part[lrow] + l_part[PM + lrow];   // both column halves
-        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_row : 0.f;
+        const float vsc = __uint_as_float((uint32_t)(127 + ev) << 23);
+        // one split: O / l; several: O unnormalised, with the row's max and sum beside it
+        const float inv = !row_ok ? 0.f : (a.splits > 1 ? vsc : vsc / l_row);
+        if (a.splits > 1 && row_ok && hf == 0) {
+            float* ml = a.part + (long long)a.splits * rows_all * D + ((long long)sp * rows_all + orow_idx) * 2;
+            ml[0] = m_run;
+            ml[1] = l_row;
+        }
         const bool folded = n_tiles > PF_FOLD;
 #pragma unroll 1
         for (int c = hf * DH; c < (hf + 1) * DH; c += 32) {
@@ -1373,7 +1393,6 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         }
     } else if (row_ok && any_fault) {
         if (tid == 0) atomicOr(lv.status, STATUS_WAIT_TIMEOUT);
-        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = hf * DH; c < (hf + 1) * DH; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
     // every copy issued must have landed, and every MMA finished, before the shared and
@@ -1399,6 +1418,33 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     if (warp == 0) t5::tmem_dealloc(tmem, 512);
 }
 
+// Rows of a split prefill: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s
+// (scores in the base-2 domain). One warp per row.
+__global__ void __launch_bounds__(256) prefill_merge(const float* part, float* out, long long rows_all, int splits,
+                                                     int D) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows_all) return;
+    const float* ml = part + (long long)splits * rows_all * D;
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[((long long)s * rows_all + row) * 2]);
+    float w[4], L = 0.f;
+    for (int s = 0; s < 4; ++s) {
+        const float m = s < splits ? ml[((long long)s * rows_all + row) * 2] : -INFINITY;
+        w[s] = (m == -INFINITY) ? 0.f : mma::ex2(m - M);
+        if (s < splits) L += w[s] * ml[((long long)s * rows_all + row) * 2 + 1];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int c = 4 * lane; c < D; c += 128) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < splits; ++s) {
+            const float4 o = *reinterpret_cast<const float4*>(part + ((long long)s * rows_all + row) * D + c);
+            acc.x += w[s] * o.x; acc.y += w[s] * o.y; acc.z += w[s] * o.z; acc.w += w[s] * o.w;
+        }
+        *reinterpret_cast<float4*>(out + row * D + c) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+}
+
 template <int NB>
 cudaError_t launch_staged_nb(const StagedArgs& a, cudaStream_t st) {
     constexpr int D = 32 * NB;
@@ -1415,8 +1461,12 @@ cudaError_t launch_staged_nb(const StagedArgs& a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         raised = true;
     }
-    const dim3 grid((unsigned)((a.C * lv.G + PM - 1) / PM), (unsigned)lv.H, (unsigned)lv.B);
+    const dim3 grid((unsigned)((a.C * lv.G + PM - 1) / PM), (unsigned)lv.H, (unsigned)(lv.B * a.splits));
     prefill_staged<NB><<<grid, SP_THREADS, sp_smem(D), st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.splits == 1) return e;
+    const long long rows_all = (long long)lv.B * a.C * lv.G * lv.H;
+    prefill_merge<<<(unsigned)((rows_all + 7) / 8), 256, 0, st>>>(a.part, a.out, rows_all, a.splits, D);
     return cudaGetLastError();
 }
 
@@ -1453,8 +1503,30 @@ size_t prefill_image_bytes(int B, int H, int D, long long max_ctx) {
     return (size_t)B * H * (size_t)((max_ctx + PN - 1) / PN) * tile_image_bytes(D);
 }
 
+size_t prefill_partial_bytes(int B, int Hq, int D, int C) {
+    return (size_t)PF_MAX_SPLITS * B * C * Hq * (D + 2) * sizeof(float);
+}
+
+// Key-range splits of the staged prefill: CTAs (one per SM) = M-tiles x H x B x splits; the
+// count that fills the last wave best, each extra split charged 1% (its pipeline start and
+// the merge), and only while every split of the first M-tile keeps 32 tiles or more.
+int prefill_splits(int B, int H, int G, int C, long long n, int num_sms) {
+    const long long ctas = (long long)((C * G + PM - 1) / PM) * H * B;
+    const long long first_tiles = (n - C + (std::min(C * G, PM) - 1) / G) / PN + 1;
+    int best = 1;
+    double best_score = -1.0;
+    for (int s = 1; s <= PF_MAX_SPLITS; ++s) {
+        if (s > 1 && first_tiles < 32LL * s) break;
+        const long long units = ctas * s;
+        const long long waves = (units + num_sms - 1) / num_sms;
+        const double score = (double)units / ((double)waves * num_sms) - 0.01 * (s - 1);
+        if (score > best_score + 1e-9) { best_score = score; best = s; }
+    }
+    return best;
+}
+
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
-                           cudaStream_t st, uint8_t* img, long long img_tiles) {
+                           cudaStream_t st, uint8_t* img, long long img_tiles, float* part, int num_sms) {
     if (img && prefill_staged_used(lv.D, C, lv.G)) {
         StagedArgs s{};
         s.lv = lv;
@@ -1465,6 +1537,8 @@ cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, flo
         s.C = C;
         s.img = img;
         s.img_tiles = img_tiles;
+        s.splits = part ? prefill_splits(lv.B, lv.H, lv.G, C, n, num_sms) : 1;
+        s.part = part;
         if (lv.D == 256) return launch_staged_nb<8>(s, st);
         if (lv.D == 128) return launch_staged_nb<4>(s, st);
         return cudaErrorInvalidValue;
