@@ -150,7 +150,9 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const float* k, c
  * (n_query_rows = n_chunk). For a prefill at head dim 128 / 256 with n_chunk * G > 128 (more
  * than one 128-row tile of query rows per kv head) the workspace holds the K~ / V~ operand
  * tiles dequantized once per (batch, kv head): 128 * head_dim bytes per position of max_ctx
- * per (batch, kv head). Otherwise it holds the per-split softmax partials of the
+ * per (batch, kv head), then room for up to 4 key-range partials of every query row
+ * (4 * batch * n_chunk * n_q_heads * (head_dim + 2) floats; the library splits the rows'
+ * key range when that fills the GPU better, and merges the partials). Otherwise it holds the per-split softmax partials of the
  * split-K decode ([OFFLOAD]: decode streams the whole attention state each step, so the
  * positions are split across the GPU and the partials merged). KVQ_ERR_NOT_BOUND before a
  * bind (the split count depends on the device's SM count). */
