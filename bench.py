@@ -103,8 +103,10 @@ def step_accounting():
     chunk = append_bytes(N_FILL, C_PF) * L_
     dec_app = sum(append_bytes(N_FILL + C_PF + s, 1) for s in range(N_DEC)) * L_
     pf = prefill_flops(N_FILL, C_PF) * L_
-    # launches: one per append; prefill one; decode = ring pass + low-bit pass + merge
-    launches = L_ * (len(fill_plan()) + 1 + 1) + L_ * N_DEC * (1 + 3)
+    # launches: one per append; the prefill builds the tile images, runs the staged kernel
+    # (its 768 M-tile CTAs split 4 ways over the key range on 148 SMs) and merges the
+    # splits; decode = ring pass + low-bit pass + merge
+    launches = L_ * (len(fill_plan()) + 1 + 3) + L_ * N_DEC * (1 + 3)
     return {"decode_bytes": dec, "fill_bytes": fill, "fill_positions": N_FILL * L_, "chunk_bytes": chunk,
             "decode_append_bytes": dec_app, "prefill_flop": pf, "launches": launches}
 
@@ -578,7 +580,8 @@ def run_kvq(args, rank, world):
         "roofline_prefill": {"bound": "tensor", "achieved": pf_tflops, "peak": peaks["bf16_tflops_sustained"],
                              "unit": "TFLOP/s", "frac": pf_tflops / peaks["bf16_tflops_sustained"], "traffic": None,
                              "peak_source": peaks["source"] + " (bf16_tflops_sustained; fp16 runs at the bf16 rate)",
-                             "kernel": "prefill_tc5, 4,096 rows over 262,080 positions, algorithmic FLOP",
+                             "kernel": "prefill_tiles + prefill_staged + prefill_merge, 4,096 rows over 262,080 "
+                                       "positions, algorithmic FLOP",
                              "algorithmic_flop_per_step": acct["prefill_flop"]},
         "cpu_baseline": cpu,
         "e2e": {"value": world * acct["decode_bytes"] / e2e_s / 1e9, "unit": "GB/s",

@@ -51,9 +51,10 @@ def test_headline_step_accounting():
     per_layer = 4 * (257984 * 2048 + (257984 - 2048) * 384 + 2048 * 544 + (32 - 1) * 2048 * 544 * 2)
     assert a["fill_bytes"] == 16 * per_layer
     assert a["fill_positions"] == 16 * 257984
-    # launches: 32 fill appends + the chunk append + the prefill per layer; each decode step
-    # appends once and launches the ring pass, the low-bit pass and the merge per layer
-    assert a["launches"] == 16 * 34 + 16 * 64 * 4
+    # launches: 32 fill appends + the chunk append + the prefill's three (tile images, staged
+    # kernel, split merge) per layer; each decode step appends once and launches the ring
+    # pass, the low-bit pass and the merge per layer
+    assert a["launches"] == 16 * 36 + 16 * 64 * 4
 
 
 def test_prefill_flop_count():
