@@ -731,6 +731,30 @@ def supplementary(dev, peaks):
     res["index_gather_2048"] = {"us": tg * 1e6, "gathered_bytes": gbytes, "gbs": gbytes / tg / 1e9,
                                 "context": n, "positions_per_kv_head": k_list,
                                 "note": "latency-bound: 3.2 MB gathered per call"}
+
+    # multi-query verify (MTP): chunks of 1, 2, 4 and 8 draft rows through the prefill entry
+    # point over the same full-length layer (the last C positions are the chunk), L2 flushed
+    # before each call; bytes = every stored row the call reads + q + out
+    verify = {}
+    for C in (1, 2, 4, 8):
+        qv = torch.randn(1, C, HQ_, D_, device=dev, generator=gen) / math.sqrt(D_)
+        ov = torch.empty_like(qv)
+        wsv = c.ensure_workspace(C)
+        tv = []
+        for i in range(8):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kvq.kvq_prefill_attention(c.handle, 0, qv, C, 1.0, ov, wsv, wsv.numel())
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                tv.append(e0.elapsed_time(e1) / 1e3)
+        tm = statistics.median(tv)
+        vbytes = decode_bytes(n) + 2 * (C - 1) * HQ_ * D_ * 4
+        verify[f"C={C}"] = {"us": tm * 1e6, "gbs": vbytes / tm / 1e9, "frac": vbytes / tm / 1e9 / peak}
+    res["multi_query_verify"] = dict(verify, note="on-the-fly tcgen05 prefill, key range split over the SMs; "
+                                                  f"context {n}")
     del c, idx
     torch.cuda.empty_cache()
 

@@ -281,11 +281,14 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache* c, int32_t n_query_rows, 
     const long long max_split = 2 * (per_unit < 1 ? 1 : per_unit) + 2;
     const int G = c->L.n_q_heads / c->L.n_kv_heads;
     *bytes = (size_t)units * max_split * partial_floats(G, c->L.head_dim) * sizeof(float);
-    // a prefill on the staged tensor-core path keeps its dequantized tile images here instead
-    if (!c->L.k_per_channel && prefill_staged_used(c->L.head_dim, n_query_rows, G)) {
-        const size_t img = prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx);
-        const size_t all = align_up(img, 256) + prefill_partial_bytes(c->L.batch, c->L.n_q_heads, c->L.head_dim,
-                                                                 n_query_rows);
+    // a tensor-core prefill keeps its key-range partials here, after the dequantized tile
+    // images on the staged path
+    if (!c->L.k_per_channel && prefill_supported(c->L.head_dim) && n_query_rows > 1) {
+        const size_t img = prefill_staged_used(c->L.head_dim, n_query_rows, G)
+                               ? align_up(prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx), 256)
+                               : 0;
+        const size_t all = img + prefill_partial_bytes(c->L.batch, c->L.n_kv_heads, c->L.n_q_heads, c->L.head_dim,
+                                                       n_query_rows);
         if (all > *bytes) *bytes = all;
     }
     return KVQ_OK;
@@ -342,7 +345,11 @@ kvq_status kvq_decode_attention_indexed(kvq_cache* c, int32_t layer, const float
 kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, int32_t n_chunk, float scale,
                                  float* out, void* ws, size_t ws_bytes, void* stream) {
     if (n_chunk < 1) return KVQ_ERR_INVALID_ARG;
-    if (c && prefill_supported(c->L.head_dim) && !c->L.k_per_channel) {
+    // Chunks of up to 4 rows (a multi-query verify) take the split-K decode kernel, one pass
+    // over the keys per row, which streams the cache at the decode's rate; longer chunks take
+    // the tcgen05 prefill, whose cost does not grow with the rows of an M-tile.
+    constexpr int DECODE_PATH_ROWS = 4;
+    if (c && prefill_supported(c->L.head_dim) && !c->L.k_per_channel && n_chunk > DECODE_PATH_ROWS) {
         // tensor-core path: validated like the split-K path, needs no workspace
         if (layer < 0 || layer >= c->L.n_layers || !q || !out || !ws) return KVQ_ERR_INVALID_ARG;
         if (!c->buf) return KVQ_ERR_NOT_BOUND;
@@ -356,12 +363,13 @@ kvq_status kvq_prefill_attention(kvq_cache* c, int32_t layer, const float* q, in
         if (ws_bytes < need) return KVQ_ERR_CAPACITY;
         const int G = c->L.n_q_heads / c->L.n_kv_heads;
         const bool staged = prefill_staged_used(c->L.head_dim, n_chunk, G);
-        if (!staged)
-            return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream));
-        const size_t img = prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim, c->L.max_ctx);
+        // the key-range partials follow the tile images (staged path) or fill the workspace
+        const size_t img = staged ? align_up(prefill_image_bytes(c->L.batch, c->L.n_kv_heads, c->L.head_dim,
+                                                                 c->L.max_ctx), 256)
+                                  : 0;
         return cuda_status(launch_prefill(layer_view(c, layer), q, scale, out, n, n_chunk, (cudaStream_t)stream,
-                                          (uint8_t*)ws, (c->L.max_ctx + 31) / 32,
-                                          (float*)((uint8_t*)ws + align_up(img, 256)), c->num_sms));
+                                          staged ? (uint8_t*)ws : nullptr, staged ? (c->L.max_ctx + 31) / 32 : 0,
+                                          (float*)((uint8_t*)ws + img), ws_bytes - img, c->num_sms));
     }
     return attention_common(c, layer, q, n_chunk, scale, out, ws, ws_bytes, stream);
 }

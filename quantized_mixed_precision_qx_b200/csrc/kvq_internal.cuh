@@ -177,14 +177,16 @@ bool prefill_supported(int D);
 // streamed by every M-tile CTA) runs when a head has more than one 128-row M-tile.
 bool prefill_staged_used(int D, int C, int G);
 size_t prefill_image_bytes(int B, int H, int D, long long max_ctx);
-// partials of a staged prefill whose M-tiles are split over the key range (Hq query heads)
-size_t prefill_partial_bytes(int B, int Hq, int D, int C);
-// img: image area of prefill_image_bytes(B, H, D, img_tiles * 32) bytes, or nullptr for the
-// on-the-fly kernel; part: prefill_partial_bytes of workspace (nullptr: no key-range splits),
-// num_sms: the device's SM count (picks the split count)
+// partials of a tensor-core prefill whose M-tiles are split over the key range (H kv heads,
+// Hq query heads, a chunk of C rows)
+size_t prefill_partial_bytes(int B, int H, int Hq, int D, int C);
+// img: image area of prefill_image_bytes(B, H, D, img_tiles * 32) bytes for the staged
+// kernel, or nullptr for the on-the-fly kernel; part: prefill_partial_bytes of workspace
+// (nullptr: no key-range splits) of part_bytes (caps the split count), num_sms: the device's
+// SM count (picks the split count)
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
                            cudaStream_t st, uint8_t* img = nullptr, long long img_tiles = 0,
-                           float* part = nullptr, int num_sms = 0);
+                           float* part = nullptr, size_t part_bytes = 0, int num_sms = 0);
 
 // One warp waits, with the bounded wait the pipelined kernels use and a limit of limit_ns,
 // on an mbarrier that nothing ever arrives on, then records the timeout in *status.

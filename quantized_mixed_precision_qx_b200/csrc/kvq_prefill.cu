@@ -42,6 +42,7 @@ constexpr float PF_RESCALE = 8.0f;
 // in tensor memory lose precision (over 100k positions the error grows past 1e-4).
 constexpr int PF_FOLD = 128;
 constexpr int PF_MAX_SPLITS = 4;   // key-range splits of a staged prefill M-tile
+constexpr int PF_OTF_MAX_SPLITS = 64;   // of an on-the-fly prefill M-tile (few rows, one wave)
 
 struct PrefillArgs {
     LayerView lv;
@@ -52,6 +53,9 @@ struct PrefillArgs {
     int C;                        // chunk rows
     int stage_half;               // bytes of one staging half (PN rows of the widest K|V row), multiple of 16
     int kbufs;                    // K~ buffers (2 when shared memory allows, else 1)
+    int splits;                   // key-range splits per M-tile (1: rows finished in place)
+    float* part;                  // splits > 1: [splits][B * C * Hq][D] unnormalised O, then
+                                  // [splits][B * C * Hq][2] (running max, row sum)
 };
 
 // shared memory: Q hi, kbufs K~ tiles, V~^T, P (all 1024-byte multiples), then the 2
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool owner = warp < OWNER_WARPS;           // owns TMEM lane / query row tid
     const int G = lv.G, H = lv.H;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = blockIdx.z / a.splits, sp = blockIdx.z % a.splits;
     const int rows_total = a.C * G;
     const int row0 = blockIdx.x * PM;
     const int r = row0 + (tid & (PM - 1));           // query row of an owner thread
@@ -328,7 +332,17 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     const SideView vside = side_view(lv, b, h, 1);
     const int W = lv.W;
     const int ring0 = W > 0 ? n - W : n;             // first position held in the ring
-    const int n_tiles = tile_limit / PN + 1;
+    // this CTA's key tiles: [t_lo, t_lo + n_tiles) of the M-tile's tiles_all (positions from
+    // tb = t_lo * PN; the host splits only when every split keeps 32 tiles or more); tile
+    // indices below count from t_lo
+    const int tiles_all = tile_limit / PN + 1;
+    const int t_lo = (int)((long long)tiles_all * sp / a.splits);
+    const int n_tiles = (int)((long long)tiles_all * (sp + 1) / a.splits) - t_lo;
+    const int tb = t_lo * PN;
+    const long long rows_all = (long long)lv.B * a.C * G * H;
+    const long long orow_idx = ((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi;
+    // where the row's O goes: the output row, or this split's partial
+    float* const orow = a.splits > 1 ? a.part + ((long long)sp * rows_all + orow_idx) * D : a.out + orow_idx * D;
     // K~ and V~ enter the MMAs scaled by 2^-ek, 2^-ev (exponents from the bounds the appends
     // keep, 0 for ordinary ranges) so that their fp16 hi + lo parts neither overflow nor lose
     // their low part to fp16's subnormal range; S and O are scaled back exactly
@@ -368,7 +382,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     // bulk copies of tile `tile`'s raw rows into staging buffer tile % 2 (issuer lane)
     int st_last[2] = {-1, -1};                       // last tile staged per buffer
     auto issue_stage = [&](int tile) {
-        const int t0 = tile * PN;
+        const int t0 = tb + tile * PN;
         const int tl = min(t0 + PN - 1, tile_limit);
         const int nm = max(0, min(tl + 1, ring0) - t0);       // rows from the low-bit store
         const int nr = (tl + 1 - t0) - nm;                    // rows from the ring
@@ -476,7 +490,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         const int tl = min(t0 + PN - 1, tile_limit);
         t = min(t, tl);
         const int nm = max(0, min(tl + 1, ring0) - t0);
-        const uint8_t* base = stage + (size_t)((t0 / PN) & 1) * 2 * SH + kv * SH;
+        const uint8_t* base = stage + (size_t)(((t0 - tb) / PN) & 1) * 2 * SH + kv * SH;
         if (t - t0 < nm) { sel = 0; return base + (size_t)(t - t0) * fm.stride; }
         sel = 1;
         return base + (size_t)nm * fm.stride + (size_t)(t - t0 - nm) * ft.stride;
@@ -489,10 +503,9 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
 
     if (owner) {
         // ======================= softmax: S(t) -> P(t), running max and sum of the row
-        float* const orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
-            const int t0 = t * PN;
+            const int t0 = tb + t * PN;
             const int sb = t & 1;
             if (!warp_wait(&s_full[sb], (t >> 1) & 1)) { set_fault(); break; }
             t5::fence_after_sync();
@@ -591,7 +604,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         constexpr int GUNITS = (PN / 8) * CHUNKS * 2;    // generic V: (8 positions, 4 channels)
         for (int t = 0; t < n_tiles; ++t) {
             if (*fault_flag) break;
-            const int t0 = t * PN;
+            const int t0 = tb + t * PN;
             // K~ buffer of this tile: free once the S MMAs of tile t - KB have read it
             const int kb = KB == 2 ? (t & 1) : 0;
             uint8_t* k_hi = k_base + (size_t)kb * 2 * PN * D * 2;
@@ -783,8 +796,14 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
     __syncthreads();
     const bool any_fault = *fault_flag != 0;
     if (owner && !any_fault) {
-        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
-        const float inv = row_ok ? __uint_as_float((uint32_t)(127 + ev) << 23) / l_run : 0.f;
+        const float vsc = __uint_as_float((uint32_t)(127 + ev) << 23);
+        // one split: O / l; several: O unnormalised, with the row's max and sum beside it
+        const float inv = !row_ok ? 0.f : (a.splits > 1 ? vsc : vsc / l_run);
+        if (a.splits > 1 && row_ok) {
+            float* ml = a.part + (long long)a.splits * rows_all * D + ((long long)sp * rows_all + orow_idx) * 2;
+            ml[0] = m_run;
+            ml[1] = l_run;
+        }
         const bool folded = n_tiles > PF_FOLD;      // a partial of earlier tiles is in orow
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
@@ -804,7 +823,6 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_tc5(PrefillArgs a) {
         }
     } else if (row_ok && any_fault) {
         if (tid == 0) atomicOr(lv.status, STATUS_WAIT_TIMEOUT);
-        float* orow = a.out + (((long long)b * a.C + ci) * (G * H) + (long long)h * G + gi) * D;
         for (int c = 0; c < D; ++c) orow[c] = __int_as_float(0x7fc00000);
     }
     if (any_fault && issuer) {
@@ -1428,18 +1446,20 @@ __global__ void __launch_bounds__(256) prefill_merge(const float* part, float* o
     const float* ml = part + (long long)splits * rows_all * D;
     float M = -INFINITY;
     for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[((long long)s * rows_all + row) * 2]);
-    float w[4], L = 0.f;
-    for (int s = 0; s < 4; ++s) {
-        const float m = s < splits ? ml[((long long)s * rows_all + row) * 2] : -INFINITY;
-        w[s] = (m == -INFINITY) ? 0.f : mma::ex2(m - M);
-        if (s < splits) L += w[s] * ml[((long long)s * rows_all + row) * 2 + 1];
+    float L = 0.f;
+    for (int s = 0; s < splits; ++s) {
+        const float m = ml[((long long)s * rows_all + row) * 2];
+        if (m != -INFINITY) L += mma::ex2(m - M) * ml[((long long)s * rows_all + row) * 2 + 1];
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     for (int c = 4 * lane; c < D; c += 128) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < splits; ++s) {
+            const float m = ml[((long long)s * rows_all + row) * 2];
+            if (m == -INFINITY) continue;
+            const float w = mma::ex2(m - M);
             const float4 o = *reinterpret_cast<const float4*>(part + ((long long)s * rows_all + row) * D + c);
-            acc.x += w[s] * o.x; acc.y += w[s] * o.y; acc.z += w[s] * o.z; acc.w += w[s] * o.w;
+            acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
         }
         *reinterpret_cast<float4*>(out + row * D + c) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
@@ -1488,8 +1508,12 @@ cudaError_t launch_prefill_nb(PrefillArgs a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         raised = true;
     }
-    const dim3 grid((unsigned)((a.C * a.lv.G + PM - 1) / PM), (unsigned)a.lv.H, (unsigned)a.lv.B);
+    const dim3 grid((unsigned)((a.C * a.lv.G + PM - 1) / PM), (unsigned)a.lv.H, (unsigned)(a.lv.B * a.splits));
     prefill_tc5<NB><<<grid, PTHREADS, smem, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.splits == 1) return e;
+    const long long rows_all = (long long)a.lv.B * a.C * a.lv.G * a.lv.H;
+    prefill_merge<<<(unsigned)((rows_all + 7) / 8), 256, 0, st>>>(a.part, a.out, rows_all, a.splits, D);
     return cudaGetLastError();
 }
 
@@ -1503,8 +1527,11 @@ size_t prefill_image_bytes(int B, int H, int D, long long max_ctx) {
     return (size_t)B * H * (size_t)((max_ctx + PN - 1) / PN) * tile_image_bytes(D);
 }
 
-size_t prefill_partial_bytes(int B, int Hq, int D, int C) {
-    return (size_t)PF_MAX_SPLITS * B * C * Hq * (D + 2) * sizeof(float);
+size_t prefill_partial_bytes(int B, int H, int Hq, int D, int C) {
+    // the staged path (several M-tiles per head) splits at most PF_MAX_SPLITS ways, the
+    // on-the-fly path (one M-tile per head) at most PF_OTF_MAX_SPLITS
+    const int max_splits = prefill_staged_used(D, C, Hq / H) ? PF_MAX_SPLITS : PF_OTF_MAX_SPLITS;
+    return (size_t)max_splits * B * C * Hq * (D + 2) * sizeof(float);
 }
 
 // Key-range splits of the staged prefill: CTAs (one per SM) = M-tiles x H x B x splits; the
@@ -1525,8 +1552,24 @@ int prefill_splits(int B, int H, int G, int C, long long n, int num_sms) {
     return best;
 }
 
+// Key-range splits of the on-the-fly prefill (C * G <= 128: one M-tile per head, few CTAs):
+// as many as fill one wave of CTAs (one per SM), up to PF_OTF_MAX_SPLITS, while every split
+// keeps 32 tiles or more.
+int prefill_otf_splits(int B, int H, int G, int C, long long n, int num_sms) {
+    const long long ctas = (long long)((C * G + PM - 1) / PM) * H * B;
+    const long long first_tiles = (n - C + (std::min(C * G, PM) - 1) / G) / PN + 1;
+    long long s = num_sms / ctas;
+    s = std::min(s, first_tiles / 32);
+    s = std::min(s, (long long)PF_OTF_MAX_SPLITS);
+    return (int)std::max(1LL, s);
+}
+
 cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, float* out, long long n, int C,
-                           cudaStream_t st, uint8_t* img, long long img_tiles, float* part, int num_sms) {
+                           cudaStream_t st, uint8_t* img, long long img_tiles, float* part, size_t part_bytes,
+                           int num_sms) {
+    // splits the partial area holds
+    const long long per_split = (long long)lv.B * C * lv.G * lv.H * (lv.D + 2) * (long long)sizeof(float);
+    const int cap = part ? (int)std::min<long long>(PF_OTF_MAX_SPLITS, (long long)(part_bytes / per_split)) : 1;
     if (img && prefill_staged_used(lv.D, C, lv.G)) {
         StagedArgs s{};
         s.lv = lv;
@@ -1537,7 +1580,7 @@ cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, flo
         s.C = C;
         s.img = img;
         s.img_tiles = img_tiles;
-        s.splits = part ? prefill_splits(lv.B, lv.H, lv.G, C, n, num_sms) : 1;
+        s.splits = cap >= 2 ? std::min(cap, prefill_splits(lv.B, lv.H, lv.G, C, n, num_sms)) : 1;
         s.part = part;
         if (lv.D == 256) return launch_staged_nb<8>(s, st);
         if (lv.D == 128) return launch_staged_nb<4>(s, st);
@@ -1550,6 +1593,8 @@ cudaError_t launch_prefill(const LayerView& lv, const float* q, float scale, flo
     a.qscale = scale * 1.4426950408889634f;
     a.n = n;
     a.C = C;
+    a.splits = cap >= 2 ? std::min(cap, prefill_otf_splits(lv.B, lv.H, lv.G, C, n, num_sms)) : 1;
+    a.part = part;
     if (lv.D == 256) return launch_prefill_nb<8>(a, st);
     if (lv.D == 128) return launch_prefill_nb<4>(a, st);
     return cudaErrorInvalidValue;

@@ -1,9 +1,11 @@
-"""GPU parity of the staged tensor-core prefill when its 128-row M-tiles are split over the key
-range (a CTA per split, partial O with the row's running max and sum, then a merge): few
-M-tiles against a long context, where the split count that best fills the SMs is the
+"""GPU parity of the tensor-core prefill when its 128-row M-tiles are split over the key range
+(a CTA per split, partial O with the row's running max and sum, then a merge). Staged kernel:
+few M-tiles against a long context, where the split count that best fills the SMs is the
 largest (4); batch 2 (the grid's batch / split index); head dims 128 and 256; formats with a
-q8_0 / bf16 ring and without one; and a context too short to split (the first M-tile must
-keep 32 tiles per split), whose rows are finished in place."""
+q8_0 / bf16 ring and without one; a context too short to split (the first M-tile must keep 32
+tiles per split), whose rows are finished in place. Verify chunks of 1 to 8 rows over a
+20,000-position context: the split-K decode kernel up to 4 rows, then the on-the-fly tcgen05
+kernel (one M-tile per kv head) split many ways."""
 import numpy as np
 import pytest
 
@@ -38,3 +40,19 @@ def test_short_context_prefill(T, C):
     q = wl.q_prefill(0, C)
     check_close(g.prefill(0, to_dev(q), 1.0).cpu().numpy(), o.prefill(0, q, 1.0), vmax,
                 f"prefill n={T} C={C}")
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("C", [1, 3, 4, 5, 8])
+def test_short_chunk_split(D, C):
+    """A multi-query verify chunk (C rows, one M-tile per kv head) over a long context: up to 4
+    rows take the split-K decode kernel (one pass per row); from 5 rows the on-the-fly tcgen05
+    kernel splits the key range over many CTAs (here up to 19 per M-tile)."""
+    T = 20000
+    wl = Workload(1, 2, 2, 12, D, T, KVRecipe("outlier"), seed=160 + C)
+    g, o = make_pair(wl, orc.Q6_0, orc.Q5_0, orc.Q8_0, 1024)
+    vmax = append_both(g, o, wl, 0, 0, T - C)
+    vmax = max(vmax, append_both(g, o, wl, 0, T - C, T))
+    q = wl.q_prefill(0, C)
+    check_close(g.prefill(0, to_dev(q), 1.0).cpu().numpy(), o.prefill(0, q, 1.0), vmax,
+                f"verify chunk C={C} D={D}")
