@@ -152,7 +152,9 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const float* k, c
  * tiles dequantized once per (batch, kv head): 128 * head_dim bytes per position of max_ctx
  * per (batch, kv head), then room for up to 4 key-range partials of every query row
  * (4 * batch * n_chunk * n_q_heads * (head_dim + 2) floats; the library splits the rows'
- * key range when that fills the GPU better, and merges the partials). Otherwise it holds the per-split softmax partials of the
+ * key range when that fills the GPU better, and merges the partials). With a single tile
+ * per kv head (n_chunk * G <= 128, n_chunk > 1) it holds up to 64 such partials per row, or
+ * the split-K partials below if those are larger. Otherwise it holds the per-split softmax partials of the
  * split-K decode ([OFFLOAD]: decode streams the whole attention state each step, so the
  * positions are split across the GPU and the partials merged). KVQ_ERR_NOT_BOUND before a
  * bind (the split count depends on the device's SM count). */
@@ -186,7 +188,10 @@ KVQ_API kvq_status kvq_decode_attention_indexed(kvq_cache* cache, int32_t layer,
  * "Engine speed and cache reuse": prompt processing with the config D cache; chunk row i
  * sits at position n - n_chunk + i and attends to positions <= its own over the
  * post-append cache). q, out: float32 [batch][n_chunk][n_q_heads][head_dim].
- * Requires 1 <= n_chunk <= n. ws: >= kvq_decode_workspace_bytes(n_chunk). */
+ * Requires 1 <= n_chunk <= n. ws: >= kvq_decode_workspace_bytes(n_chunk). Chunks of up to 4
+ * rows (a multi-query verify) run on the split-K decode kernels, one pass over the keys per
+ * row; longer chunks at head dim 128 / 256 on the tensor-core (tcgen05) prefill, which may
+ * split each 128-row tile of query rows over the key range and merge the parts. */
 KVQ_API kvq_status kvq_prefill_attention(kvq_cache* cache, int32_t layer, const float* q, int32_t n_chunk,
                                  float scale, float* out, void* ws, size_t ws_bytes, void* stream);
 
