@@ -24,6 +24,7 @@
 #include "kvq_rowio.cuh"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace kvq {
 namespace {
@@ -95,11 +96,15 @@ __device__ __forceinline__ void round_codes(const float (&x)[CPL], float d, floa
 // pack CPL codes (bits below W0 into plane 0, the next W1 bits into plane 1) and store
 template <int CPL, int W0, int W1>
 __device__ __forceinline__ void pack_store(uint8_t* p0, uint8_t* p1, int lane, const uint32_t (&u)[CPL]) {
-    uint64_t v0 = 0, v1 = 0;
+    // 32-bit accumulators unless a lane's plane bits need 64
+    using A0 = typename std::conditional<(CPL * W0 > 32), uint64_t, uint32_t>::type;
+    using A1 = typename std::conditional<(CPL * W1 > 32), uint64_t, uint32_t>::type;
+    A0 v0 = 0;
+    A1 v1 = 0;
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
-        v0 |= (uint64_t)(u[j] & ((1u << W0) - 1)) << (j * W0);
-        if constexpr (W1 > 0) v1 |= (uint64_t)(u[j] >> W0) << (j * W1);
+        v0 |= (A0)(u[j] & ((1u << W0) - 1)) << (j * W0);
+        if constexpr (W1 > 0) v1 |= (A1)(u[j] >> W0) << (j * W1);
     }
     // a row of D = 32 * CPL channels has CPL blocks
     store_plane_bits<CPL>(p0, CPL, lane, W0, v0);
@@ -215,15 +220,14 @@ __device__ __forceinline__ void store_low(uint8_t* row, const RowFmt& f, const f
 // Raise the cache's per-head bounds (float bits of non-negative values compare as unsigned
 // integers) to this warp's; the read first keeps the atomic off the common path.
 __device__ __forceinline__ void publish_bounds(uint32_t* st, Bounds bd) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        bd.stored = fmaxf(bd.stored, __shfl_xor_sync(0xffffffffu, bd.stored, off));
-        bd.deq = fmaxf(bd.deq, __shfl_xor_sync(0xffffffffu, bd.deq, off));
-    }
+    // warp maxima of the two bounds (non-negative, so their bits order as unsigned integers;
+    // a NaN bound, which only a NaN input makes, orders above every finite one)
+    const uint32_t s_max = __reduce_max_sync(0xffffffffu, __float_as_uint(bd.stored));
+    const uint32_t d_max = __reduce_max_sync(0xffffffffu, __float_as_uint(bd.deq));
     if ((threadIdx.x & 31) == 0) {
         // margin for the fp32 rounding of dequantized values
-        const uint32_t u0 = __float_as_uint(bd.stored * 1.0009765625f);
-        const uint32_t u1 = __float_as_uint(bd.deq * 1.0009765625f);
+        const uint32_t u0 = __float_as_uint(__uint_as_float(s_max) * 1.0009765625f);
+        const uint32_t u1 = __float_as_uint(__uint_as_float(d_max) * 1.0009765625f);
         if (u0 > __ldcg(st)) atomicMax(st, u0);
         if (u1 > __ldcg(st + 1)) atomicMax(st + 1, u1);
     }
@@ -272,21 +276,29 @@ __device__ __forceinline__ void kivi_enter(const LayerView& lv, uint32_t unit, l
     }
 }
 
+// Ring slot arithmetic without a division: q = floor(x / W) = (x * m) >> 32 + s for x < 2^31,
+// with s = ceil(log2 W) and m = ceil(2^(32 + s) / W) (Granlund and Montgomery's division by an
+// invariant integer; the error term stays below 1 / W for 31-bit x), and n mod W from the host.
+struct RingDiv {
+    unsigned long long m;
+    uint32_t s;
+    uint32_t n_mod_w;
+};
+
 template <int CPL>
 __global__ void __launch_bounds__(32 * WARPS_PER_CTA)
 append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C,
-              uint32_t kivi_done) {
+              uint32_t kivi_done, RingDiv rd) {
     const int lane = threadIdx.x & 31;
-    // item order: (b, i, h, kv) so consecutive warps read consecutive input rows; the host
-    // keeps C * B * H * 2 below 2^32 and positions below 2^31
-    const uint32_t item = blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-    const uint32_t per_pos = 2u * (uint32_t)lv.H;
-    const uint32_t row = item / per_pos;                 // b * C + i
-    if (row >= C * (uint32_t)lv.B) return;
-    const uint32_t kv = item & 1u;
-    const uint32_t h = (item - row * per_pos) >> 1;
-    const uint32_t b = row / C;
-    const uint32_t i = row - b * C;
+    // warp = one row: position i of the append (consecutive warps, consecutive positions of the
+    // same (b, h, K|V) region), blockIdx.y = 2 h + kv, blockIdx.z = b; the host keeps
+    // positions below 2^31
+    const uint32_t i = blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+    if (i >= C) return;
+    const uint32_t kv = blockIdx.y & 1u;
+    const uint32_t h = blockIdx.y >> 1;
+    const uint32_t b = blockIdx.z;
+    const uint32_t row = b * C + i;
     const int D = lv.D;
     const float* src = (kv ? v : k) + ((long long)row * lv.H + h) * D;
     const RowFmt fl = kv ? lv.fmt[1] : lv.fmt[0];   // by value: no pointer into the parameters
@@ -319,8 +331,9 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     }
     // ends inside the window: evict the slot's old occupant, then take the slot
     uint8_t* ring = lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region;
-    const uint32_t im = i % W;
-    const uint32_t slot = (n % W + im) % W;
+    const uint32_t im = i - W * (uint32_t)(((unsigned long long)i * rd.m) >> (32 + rd.s));   // i mod W
+    uint32_t slot = rd.n_mod_w + im;                                                       // (n + i) mod W
+    if (slot >= W) slot -= W;
     uint8_t* srow = ring + (long long)slot * lv.tail.stride;
     // old occupant: the position in [n - W, n) congruent to p = n + i modulo W
     const long long q = (long long)n - W + im;
@@ -477,10 +490,17 @@ __global__ void calibrate_kernel(LayerView lv, const float* __restrict__ k, cons
 
 cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, long long n, int C,
                           cudaStream_t st) {
-    const long long items = (long long)C * lv.B * lv.H * 2;
-    if (items >= (1LL << 32) - WARPS_PER_CTA || n + C > (1LL << 31)) return cudaErrorInvalidValue;
-    const unsigned grid = (unsigned)((items + WARPS_PER_CTA - 1) / WARPS_PER_CTA);
+    if (n + C > (1LL << 31) || lv.B > 65535 || 2LL * lv.H > 65535) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)((C + WARPS_PER_CTA - 1) / WARPS_PER_CTA), (unsigned)(2 * lv.H), (unsigned)lv.B);
     const dim3 block(32 * WARPS_PER_CTA);
+    RingDiv rd{0, 0, 0};
+    if (lv.W > 0) {
+        uint32_t sh = 0;
+        while ((1LL << sh) < lv.W) ++sh;
+        rd.s = sh;
+        rd.m = (unsigned long long)((((unsigned __int128)1 << (32 + sh)) + (unsigned)lv.W - 1) / (unsigned)lv.W);
+        rd.n_mod_w = (uint32_t)(n % lv.W);
+    }
     const uint32_t n32 = (uint32_t)n, C32 = (uint32_t)C;
     uint32_t done = 0;
     if (lv.kivi) {
@@ -506,10 +526,10 @@ cudaError_t launch_append(const LayerView& lv, const float* k, const float* v, l
         }
     }
     switch (lv.D / 32) {
-        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
-        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
-        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
-        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done); break;
+        case 1: append_kernel<1><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done, rd); break;
+        case 2: append_kernel<2><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done, rd); break;
+        case 4: append_kernel<4><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done, rd); break;
+        case 8: append_kernel<8><<<grid, block, 0, st>>>(lv, k, v, n32, C32, done, rd); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
