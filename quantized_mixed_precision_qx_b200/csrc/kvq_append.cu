@@ -217,19 +217,25 @@ __device__ __forceinline__ void store_low(uint8_t* row, const RowFmt& f, const f
     bd.add(b, b * smax);
 }
 
-// Raise the cache's per-head bounds (float bits of non-negative values compare as unsigned
-// integers) to this warp's; the read first keeps the atomic off the common path.
-__device__ __forceinline__ void publish_bounds(uint32_t* st, Bounds bd) {
-    // warp maxima of the two bounds (non-negative, so their bits order as unsigned integers;
-    // a NaN bound, which only a NaN input makes, orders above every finite one)
+// Raise the cache's per-head bounds to the maxima of the values a CTA of the append kernel
+// stored (its warps share one (b, h, K|V)). Float bits of non-negative values order as
+// unsigned integers (a NaN bound, which only a NaN input makes, orders above every finite
+// one); the warps' maxima meet in shared memory and one thread raises the bounds with
+// non-returning atomics, so no warp waits on a read of the bounds.
+__device__ __forceinline__ void publish_bounds_cta(uint32_t* st, Bounds bd, uint32_t (*sb)[2]) {
     const uint32_t s_max = __reduce_max_sync(0xffffffffu, __float_as_uint(bd.stored));
     const uint32_t d_max = __reduce_max_sync(0xffffffffu, __float_as_uint(bd.deq));
-    if ((threadIdx.x & 31) == 0) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) { sb[warp][0] = s_max; sb[warp][1] = d_max; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = 0, c = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { a = max(a, sb[w][0]); c = max(c, sb[w][1]); }
         // margin for the fp32 rounding of dequantized values
-        const uint32_t u0 = __float_as_uint(__uint_as_float(s_max) * 1.0009765625f);
-        const uint32_t u1 = __float_as_uint(__uint_as_float(d_max) * 1.0009765625f);
-        if (u0 > __ldcg(st)) atomicMax(st, u0);
-        if (u1 > __ldcg(st + 1)) atomicMax(st + 1, u1);
+        const uint32_t u0 = __float_as_uint(__uint_as_float(a) * 1.0009765625f);
+        const uint32_t u1 = __float_as_uint(__uint_as_float(c) * 1.0009765625f);
+        if (u0) atomicMax(st, u0);
+        if (u1) atomicMax(st + 1, u1);
     }
 }
 
@@ -285,19 +291,14 @@ struct RingDiv {
     uint32_t n_mod_w;
 };
 
+// One row of an append (warp-wide): quantize-on-append, ring eviction, requantization.
+// Returns this lane's bounds of the values it stored (zero for per-channel K rows that only
+// enter the pending buffer).
 template <int CPL>
-__global__ void __launch_bounds__(32 * WARPS_PER_CTA)
-append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C,
-              uint32_t kivi_done, RingDiv rd) {
-    const int lane = threadIdx.x & 31;
-    // warp = one row: position i of the append (consecutive warps, consecutive positions of the
-    // same (b, h, K|V) region), blockIdx.y = 2 h + kv, blockIdx.z = b; the host keeps
-    // positions below 2^31
-    const uint32_t i = blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
-    if (i >= C) return;
-    const uint32_t kv = blockIdx.y & 1u;
-    const uint32_t h = blockIdx.y >> 1;
-    const uint32_t b = blockIdx.z;
+__device__ __forceinline__ Bounds append_row(const LayerView& lv, const float* __restrict__ k,
+                                             const float* __restrict__ v, uint32_t n, uint32_t C,
+                                             uint32_t kivi_done, const RingDiv& rd, uint32_t i, uint32_t kv,
+                                             uint32_t h, uint32_t b, int lane) {
     const uint32_t row = b * C + i;
     const int D = lv.D;
     const float* src = (kv ? v : k) + ((long long)row * lv.H + h) * D;
@@ -305,8 +306,6 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     uint8_t* main = lv.main[kv] + (long long)(b * lv.H + h) * lv.main_region[kv];
     const float* s = lv.kvarn ? lv.scales + ((long long)(b * lv.H + h) * 2 + kv) * D : nullptr;
     const uint32_t p = n + i;
-
-    uint32_t* st = lv.stats + ((long long)(b * lv.H + h) * 2 + kv) * 2;
     const bool kivi = lv.kivi && kv == 0;            // per-channel K
     const uint32_t unit = b * lv.H + h;
     Bounds bd;
@@ -314,20 +313,18 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     load_row_f32<CPL>(src, lane, x);
 
     if (lv.W == 0) {
-        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, x); return; }
+        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, x); return bd; }
         store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, x, bd);
-        publish_bounds(st, bd);
-        return;
+        return bd;
     }
     const uint32_t W = (uint32_t)lv.W;
     if (i + W < C) {
         // enters and leaves the window inside this append: tail rounding, then low-bit
         float t[CPL];
         tail_round<CPL>(lv.tail, x, t);
-        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, t); return; }
+        if (kivi) { kivi_enter<CPL>(lv, unit, p, kivi_done, lane, t); return bd; }
         store_low<CPL>(main + (long long)p * fl.stride, fl, s, lane, t, bd);
-        publish_bounds(st, bd);
-        return;
+        return bd;
     }
     // ends inside the window: evict the slot's old occupant, then take the slot
     uint8_t* ring = lv.ring[kv] + (long long)(b * lv.H + h) * lv.ring_region;
@@ -347,7 +344,28 @@ append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict
     __syncwarp();
     const float rb = store_row<CPL>(srow, lv.tail, lane, x);   // ring rows hold raw values
     bd.add(rb, rb);
-    publish_bounds(st, bd);
+    return bd;
+}
+
+// 6 CTAs (48 warps) per SM: the kernel is issue-bound, and the extra warps hide more latency
+// than the few registers they cost (a handful of spills at 40 registers) take back
+template <int CPL>
+__global__ void __launch_bounds__(32 * WARPS_PER_CTA, 6)
+append_kernel(LayerView lv, const float* __restrict__ k, const float* __restrict__ v, uint32_t n, uint32_t C,
+              uint32_t kivi_done, RingDiv rd) {
+    const int lane = threadIdx.x & 31;
+    // warp = one row: position i of the append (consecutive warps, consecutive positions of the
+    // same (b, h, K|V) region), blockIdx.y = 2 h + kv, blockIdx.z = b; the host keeps
+    // positions below 2^31
+    const uint32_t i = blockIdx.x * WARPS_PER_CTA + (threadIdx.x >> 5);
+    const uint32_t kv = blockIdx.y & 1u;
+    const uint32_t h = blockIdx.y >> 1;
+    const uint32_t b = blockIdx.z;
+    uint32_t* st = lv.stats + ((long long)(b * lv.H + h) * 2 + kv) * 2;
+    __shared__ uint32_t sb[WARPS_PER_CTA][2];
+    Bounds bd;
+    if (i < C) bd = append_row<CPL>(lv, k, v, n, C, kivi_done, rd, i, kv, h, b, lane);
+    publish_bounds_cta(st, bd, sb);   // every thread of the CTA takes part
 }
 
 // Per-channel K, groups completed by an append of C positions to a cache of n0: one CTA per
