@@ -1293,6 +1293,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         const uint32_t idesc_s2 = t5::idesc_f16(PM, 2 * PN);
         const uint32_t idesc_o = t5::idesc_f16(PM, D);
         const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
+        // buffer descriptors: the base's plus the buffer offset in the 16-byte start-address
+        // field (shared-memory addresses stay below 2^18, inside the field)
+        const uint64_t dk_base = t5::desc_sw128(t5::smem_addr(kbuf));
+        const uint64_t dv_base = t5::desc_sw64(t5::smem_addr(vbuf));
         // S' = [Q hi K~hi | Q hi K~lo] in TMEM columns [0, 2 PN), S'' = Q lo K~hi in
         // [3 PN, 4 PN): the large products accumulate alone; the owners add the three. The short
         // S'' MMAs go first, so the queue holds the long ones when the issue returns.
@@ -1302,7 +1306,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             if (okk && t >= 1) okk = poll_wait(s_empty, (t - 1) & 1);   // the owners have read S(t - 1)
             if (!okk) return false;
             t5::fence_after_sync();
-            const uint64_t dk0 = t5::desc_sw128(t5::smem_addr(kbuf + (size_t)kb * KT_BYTES));
+            const uint64_t dk0 = dk_base + (uint64_t)((kb * KT_BYTES) >> 4);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
@@ -1319,9 +1323,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             s_last = t;
             return true;
         };
+        // (no fault-flag poll in this loop: every wait is bounded and a fault ends it there)
         bool ok = issue_s(0);
         for (int t = 0; ok && t < n_tiles; ++t) {
-            if (*fault_flag) break;
             if (t + 1 < n_tiles) {
                 ok = issue_s(t + 1);
                 if (!ok) break;
@@ -1330,7 +1334,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             if (ok) ok = poll_wait(&v_full[t & 1], (t >> 1) & 1);
             if (!ok) break;
             t5::fence_after_sync();
-            const uint64_t dvh0 = t5::desc_sw64(t5::smem_addr(vbuf + (size_t)(t & 1) * VT_BYTES));
+            const uint64_t dvh0 = dv_base + (uint64_t)(((t & 1) * VT_BYTES) >> 4);
             const uint64_t dvl0 = dvh0 + (uint64_t)((D * PN * 2) >> 4);
             // A operand (P hi / lo) from TMEM: 8 columns per 16-position k-step
 #pragma unroll
