@@ -994,11 +994,13 @@ struct StagedArgs {
 // Warp roles of the staged kernel: 8 softmax / epilogue warps own the 128 query rows in pairs
 // (warps w and w + 4 share TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, one row per lane: both
 // compute the row's running max from all of S, each turns its half of the tile's columns
-// into P and handles its half of the O columns), one warp whose lane 0 issues the MMAs and
-// one whose lane 0 issues the bulk copies. MMA issue stalls while the tensor pipe's short
-// queue is full, so the issuing thread does nothing else that could let the queue run dry.
+// into P and handles its half of the O columns), two warps whose lane 0 issue MMAs (one the S'
+// and P V~ MMAs, the other the S'' MMAs: an MMA occupies its issuing thread for ~50 cycles
+// whatever its size, so narrow MMAs from two threads overlap where one thread's would queue)
+// and one whose lane 0 issues the bulk copies. MMA issue stalls while the tensor pipe's short
+// queue is full, so the issuing threads do nothing else that could let the queue run dry.
 constexpr int SP_OWNERS = 8;
-constexpr int SP_THREADS = 32 * (SP_OWNERS + 2);
+constexpr int SP_THREADS = 32 * (SP_OWNERS + 3);
 constexpr int SP_KBUF = 3;                                 // K~ buffers: fetched two tiles ahead
 __host__ __device__ constexpr size_t sp_smem(int D) {
     return 1024 /* alignment slack */ + (size_t)PM * D * 2 /* Q hi */ + SP_KBUF * 2 * (size_t)PN * D * 2 /* K~ */ +
@@ -1051,6 +1053,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     const bool owner = warp < SP_OWNERS;
     const bool issuer = warp == SP_OWNERS && lane == 0;
     const bool copier = warp == SP_OWNERS + 1 && lane == 0;
+    const bool issuer2 = warp == SP_OWNERS + 2 && lane == 0;   // the S'' MMAs
     const int hf = (warp >> 2) & 1;                  // owner column half
     const int lrow = 32 * (warp & 3) + lane;         // owner's row in the M-tile
     const int G = lv.G, H = lv.H;
@@ -1084,13 +1087,13 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
     if (tid == 0) {
         for (int i = 0; i < SP_KBUF; ++i) {
             mma::mbar_init(&k_full[i], 1);
-            mma::mbar_init(&k_empty[i], 1);
+            mma::mbar_init(&k_empty[i], 2);          // both MMA threads commit
         }
         for (int i = 0; i < 2; ++i) {
             mma::mbar_init(&v_full[i], 1);
             mma::mbar_init(&v_empty[i], 1);
         }
-        mma::mbar_init(s_full, 1);
+        mma::mbar_init(s_full, 2);                   // both MMA threads commit
         mma::mbar_init(s_empty, SP_OWNERS);
         mma::mbar_init(p_full, SP_OWNERS);
         mma::mbar_init(o_done, 1);
@@ -1184,7 +1187,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
 
     float m_run = -INFINITY, l_run = 0.f;            // l_run: this warp's column half
     float gcorr = 1.f;
-    int s_last = -1, o_last = -1;
+    int s_last = -1, o_last = -1, s2_last = -1;
 
     if (owner) {
         // ======================= softmax: S(t) -> P(t), running max and sum of the row
@@ -1289,7 +1292,6 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         // ======================= MMA issue
         // Pipe order: S(t + 1), then O(t) once P(t) is written; the softmax of tile t runs
         // while S(t + 1) executes.
-        const uint32_t idesc_s = t5::idesc_f16(PM, PN);
         const uint32_t idesc_s2 = t5::idesc_f16(PM, 2 * PN);
         const uint32_t idesc_o = t5::idesc_f16(PM, D);
         const uint64_t dq0 = t5::desc_sw128(t5::smem_addr(q_hi));
@@ -1297,9 +1299,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
         // field (shared-memory addresses stay below 2^18, inside the field)
         const uint64_t dk_base = t5::desc_sw128(t5::smem_addr(kbuf));
         const uint64_t dv_base = t5::desc_sw64(t5::smem_addr(vbuf));
-        // S' = [Q hi K~hi | Q hi K~lo] in TMEM columns [0, 2 PN), S'' = Q lo K~hi in
-        // [3 PN, 4 PN): the large products accumulate alone; the owners add the three. The short
-        // S'' MMAs go first, so the queue holds the long ones when the issue returns.
+        // S' = [Q hi K~hi | Q hi K~lo] in TMEM columns [0, 2 PN) from this thread, S'' = Q lo K~hi
+        // in [3 PN, 4 PN) from the other MMA thread: the large products accumulate alone; the
+        // owners add the three once both threads have committed.
         auto issue_s = [&](int t) -> bool {
             const int kb = t % SP_KBUF;
             bool okk = poll_wait(&k_full[kb], (t / SP_KBUF) & 1);
@@ -1307,11 +1309,6 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             if (!okk) return false;
             t5::fence_after_sync();
             const uint64_t dk0 = dk_base + (uint64_t)((kb * KT_BYTES) >> 4);
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
-                t5::mma_f16_ts(t_s3, t_qlo + 8 * k, dk0 + dkk, idesc_s, k > 0);
-            }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t dq = (uint64_t)(((k >> 2) * PM * 128 + (k & 3) * 32) >> 4);
@@ -1355,6 +1352,28 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             t5::mma_commit(o_done);
             t5::mma_commit(&v_empty[t & 1]);
             o_last = t;
+        }
+        if (!ok) set_fault();
+    } else if (issuer2) {
+        // ======================= the S'' MMAs of every tile, beside the other MMA thread's
+        const uint32_t idesc_s = t5::idesc_f16(PM, PN);
+        const uint64_t dk_base = t5::desc_sw128(t5::smem_addr(kbuf));
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int kb = t % SP_KBUF;
+            ok = poll_wait(&k_full[kb], (t / SP_KBUF) & 1);
+            if (ok && t >= 1) ok = poll_wait(s_empty, (t - 1) & 1);   // the owners have read S(t - 1)
+            if (!ok) break;
+            t5::fence_after_sync();
+            const uint64_t dk0 = dk_base + (uint64_t)((kb * KT_BYTES) >> 4);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t dkk = (uint64_t)(((k >> 2) * 2 * PN * 128 + (k & 3) * 32) >> 4);
+                t5::mma_f16_ts(t_s3, t_qlo + 8 * k, dk0 + dkk, idesc_s, k > 0);
+            }
+            t5::mma_commit(s_full);
+            t5::mma_commit(&k_empty[kb]);
+            s2_last = t;
         }
         if (!ok) set_fault();
     } else if (copier) {
@@ -1424,6 +1443,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1) prefill_staged(StagedArgs a) {
             if (k_last[i] >= 0) mma::mbar_wait(&k_full[i], (k_last[i] / SP_KBUF) & 1, 50000000ull);
         for (int i = 0; i < 2; ++i)
             if (v_last[i] >= 0) mma::mbar_wait(&v_full[i], (v_last[i] >> 1) & 1, 50000000ull);
+    }
+    if (issuer2 && s2_last >= 0) {   // this thread's last commits must land too
+        mma::mbar_wait(s_full, s2_last & 1, 50000000ull);
+        mma::mbar_wait(&k_empty[s2_last % SP_KBUF], (s2_last / SP_KBUF) & 1, 50000000ull);
     }
     if (issuer) {   // the later commits of each group too (their arrivals must land first)
         if (s_last >= 0) {
