@@ -3,8 +3,16 @@
 // The chunk's C rows were just appended at positions n - C .. n - 1; chunk row i attends
 // to positions t <= n - C + i of the post-append cache (low-bit rows below the window,
 // ring rows inside it). QK^T and PV are dense contractions, so they run as tcgen05 MMAs
-// with fp32 accumulators in tensor memory:
+// with fp32 accumulators in tensor memory. Two kernels:
+//   - prefill_staged (below, with prefill_tiles): a head with more than one 128-row M-tile;
+//     each K~ / V~ tile is dequantized once per head into a workspace image that every M-tile
+//     CTA of the head streams;
+//   - prefill_tc5 (this part): one M-tile per head (short chunks); each CTA dequantizes its
+//     own tiles.
+// Either kernel may split each M-tile's key range over several CTAs (partial O with the
+// row's running max and sum) when that fills the GPU better; prefill_merge combines them.
 //
+// prefill_tc5:
 //   CTA   = 128 query rows of one (batch, kv head): row r = chunk row * G + head in group,
 //           TMEM lane r. 16 warps in three roles that signal each other through mbarriers:
 //           warps 0-3 own one row per thread (softmax, epilogue), warps 4-14 dequantize,
@@ -20,7 +28,7 @@
 //   tile overlaps the MMAs and the softmax of the previous one; the raw rows of tile t + 2
 //   are fetched by bulk copies into a staging buffer as soon as tile t is dequantized.
 //
-// Shared memory (head_dim D = 32 NB): Q hi 128 x D x 2 B (Q lo lives in TMEM), K~ hi/lo
+// Shared memory of prefill_tc5 (head_dim D = 32 NB): Q hi 128 x D x 2 B (Q lo lives in TMEM), K~ hi/lo
 // 2 x 32 x D x 2 B per K~ tile (K-major, 128-byte swizzle), V~^T hi/lo 2 x D x 32 x 2 B and
 // P hi/lo 2 x 128 x 32 x 2 B (K-major, 64-byte swizzle), 2 staging buffers of 2 x 32 raw rows
 // (sized by the widest row format).
