@@ -734,7 +734,8 @@ def supplementary(dev, peaks):
 
     # multi-query verify (MTP): chunks of 1, 2, 4 and 8 draft rows through the prefill entry
     # point over the same full-length layer (the last C positions are the chunk), L2 flushed
-    # before each call; bytes = every stored row the call reads + q + out
+    # before each call; bytes = every stored row once (the algorithmic minimum: chunks of up to
+    # 4 rows actually read the rows once per row) + q + out
     verify = {}
     for C in (1, 2, 4, 8):
         qv = torch.randn(1, C, HQ_, D_, device=dev, generator=gen) / math.sqrt(D_)
